@@ -163,6 +163,14 @@ MX_API mx_status mx_quant_weight(const void* w, int N, int K, void* codes, void*
  * size includes the quantised activations (M x K code bytes and M x K/32
  * scale bytes, each rounded up to 256 bytes).  Returns 256 when no sm_100
  * device is current.
+ *
+ * The contract follows the scratch of the vLLM DeepSeek-V4 mono runner page
+ * (MonoRunner.scratch): caller-visible device scratch per problem shape,
+ * zero-filled when first allocated, allocated on an eager call and never
+ * while a stream is being captured (the runner raises an error if a width is
+ * first reached inside a capture), so that captured launches see only
+ * pointers.  Its arrival counters reset themselves, like the runner's
+ * kernel-advanced epoch words, so the same workspace serves every replay.
  */
 MX_API size_t mx_gemm_workspace_size(int M, int N, int K, mx_a_fmt a_fmt, mx_b_fmt b_fmt, mx_epi epi);
 
@@ -233,6 +241,11 @@ MX_API const char* mx_status_string(mx_status s);
  * mx_workspace_status -- synchronises `stream`, reads the workspace status
  * word and returns MX_OK if it is zero, MX_ERR_TIMEOUT if a kernel gave up on
  * a bounded wait (the word is then cleared), MX_ERR_CUDA on a CUDA error.
+ * The word is the first 4 bytes of the workspace; kernels only OR bits into
+ * it.  It plays the part of the status words in the vLLM DeepSeek-V4 mono
+ * runner page's device mailbox (MonoRunner's epoch tensor: an epoch, a mark
+ * per CTA and counters that the kernels themselves advance), read back on
+ * the host between launches rather than by a later kernel.
  */
 MX_API mx_status mx_workspace_status(void* workspace, void* stream);
 

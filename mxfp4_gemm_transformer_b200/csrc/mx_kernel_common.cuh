@@ -48,8 +48,12 @@ __device__ __forceinline__ bool wait_bar_final(uint64_t* bar, uint32_t parity, u
 
 __device__ __forceinline__ float sigmoid_mul(float v, float t)
 {
-    // v * sigmoid(t) = v / (1 + e^-t)
-    return __fdividef(v, 1.0f + __expf(-t));
+    // v * sigmoid(t) with z = e^-|t| in (0, 1]: v / (1 + z) for t >= 0 and
+    // v z / (1 + z) for t < 0, so nothing overflows and the divisor stays in
+    // [1, 2].  z = 2^(-|t| log2 e) keeps subnormal values, so the far negative
+    // tail (t < -87, where e^t is below fp32's normal range) still gives v e^t.
+    const float z = ex2_approx(-fabsf(t) * 1.4426950408889634f);
+    return __fdividef(t >= 0.0f ? v : v * z, 1.0f + z);
 }
 
 // 0.5 v (1 + tanh(u)) == v * sigmoid(2u), u = sqrt(2/pi) (v + 0.044715 v^3)

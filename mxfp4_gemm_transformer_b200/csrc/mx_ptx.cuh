@@ -20,6 +20,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// 2^x by the hardware approximation, without flushing subnormal results to
+// zero (the .ftz form would).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---- mbarrier ------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

@@ -37,6 +37,39 @@ def build() -> str:
     return os.path.join(_HERE, "_mxref.so")
 
 
+def _signatures():
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    D = ctypes.c_double
+    U = ctypes.c_uint
+    Z = ctypes.c_size_t
+    return [
+        ("mxr_e4m3_value", D, [U]), ("mxr_e2m1_value", D, [U]), ("mxr_e8m0_value", D, [U]),
+        ("mxr_rne_e4m3", U, [D]), ("mxr_rne_e2m1", U, [D]),
+        ("mxr_e8m0_for_amax", U, [D, D]),
+        ("mxr_quant_act_e8m0", None, [P, I, I, P, P]),
+        ("mxr_quant_f32_row", None, [P, I, I, P, P]),
+        ("mxr_quant_w_e4m3_32x32", None, [P, I, I, P, P]),
+        ("mxr_quant_w_e2m1_1x32", None, [P, I, I, P, P]),
+        ("mxr_gemm", None, [P, P, I, P, P, I, P, I, I, I, I, P, P, P]),
+        ("mxr_gelu_tanh", D, [D]), ("mxr_silu", D, [D]), ("mxr_silu_grad", D, [D]),
+        ("mxr_bf16_rne", U, [D]), ("mxr_round_bf16", None, [P, Z, P]),
+        ("mxr_add_bf16", None, [P, P, Z, P]),
+        ("mxr_rmsnorm_bf16", None, [P, P, I, I, D, P]),
+    ]
+
+
+def load_library(path: str):
+    """ctypes handle of an oracle library built from mxref.c (the tests also
+    load copies with a planted mistake, to show that the pins catch it)."""
+    L = ctypes.CDLL(path)
+    for name, res, args in _signatures():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
 def lib():
     global _LIB
     if _LIB is None:
@@ -44,29 +77,7 @@ def lib():
         src = os.path.join(_HERE, "mxref.c")
         if not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(src):
             build()
-        L = ctypes.CDLL(path)
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        D = ctypes.c_double
-        U = ctypes.c_uint
-        for name, res, args in [
-            ("mxr_e4m3_value", D, [U]), ("mxr_e2m1_value", D, [U]), ("mxr_e8m0_value", D, [U]),
-            ("mxr_rne_e4m3", U, [D]), ("mxr_rne_e2m1", U, [D]),
-            ("mxr_e8m0_for_amax", U, [D, D]),
-            ("mxr_quant_act_e8m0", None, [P, I, I, P, P]),
-            ("mxr_quant_f32_row", None, [P, I, I, P, P]),
-            ("mxr_quant_w_e4m3_32x32", None, [P, I, I, P, P]),
-            ("mxr_quant_w_e2m1_1x32", None, [P, I, I, P, P]),
-            ("mxr_gemm", None, [P, P, I, P, P, I, P, I, I, I, I, P, P, P]),
-            ("mxr_gelu_tanh", D, [D]), ("mxr_silu", D, [D]),
-            ("mxr_bf16_rne", U, [D]), ("mxr_round_bf16", None, [P, ctypes.c_size_t, P]),
-            ("mxr_add_bf16", None, [P, P, ctypes.c_size_t, P]),
-            ("mxr_rmsnorm_bf16", None, [P, P, I, I, D, P]),
-        ]:
-            f = getattr(L, name)
-            f.restype = res
-            f.argtypes = args
-        _LIB = L
+        _LIB = load_library(path)
     return _LIB
 
 
@@ -298,7 +309,25 @@ def silu(v: float) -> float:
     return lib().mxr_silu(v)
 
 
+def silu_grad(v: float) -> float:
+    """The SiLU derivative the SwiGLU tolerance term uses."""
+    return lib().mxr_silu_grad(v)
+
+
+# Absolute floor of the bf16 output rounding: below bf16's normal range
+# (2^-126) its values are 2^-133 apart, so the relative 2^-8 |y| no longer
+# bounds the rounding of the output.
+BF16_FLOOR = 2.0 ** -133
+
+
+def tolerance_bound(y_ref, t_ref):
+    """2^-8 |y| (the bf16 output rounding, with its subnormal floor) + 1e-5 T
+    (fp32 accumulation-order slack)."""
+    return 2.0 ** -8 * np.abs(y_ref) + 1e-5 * t_ref + BF16_FLOOR
+
+
 def within_tolerance(y_gpu, y_ref, t_ref):
-    """Acceptance bound |y_gpu - y| <= 2^-8 |y| + 1e-5 T, elementwise."""
+    """Acceptance bound |y_gpu - y| <= 2^-8 |y| + 1e-5 T (+ 2^-133 below the
+    bf16 normal range), elementwise."""
     y_gpu = np.asarray(y_gpu, np.float64)
-    return np.abs(y_gpu - y_ref) <= 2.0 ** -8 * np.abs(y_ref) + 1e-5 * t_ref
+    return np.abs(y_gpu - y_ref) <= tolerance_bound(y_ref, t_ref)

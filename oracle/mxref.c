@@ -431,6 +431,15 @@ static double gelu_tanh(double v)
 
 static double silu(double v) { return v / (1.0 + exp(-v)); }
 
+/* d/dv silu(v) = sigma(v) (1 + v (1 - sigma(v))), sigma(v) = 1 / (1 + e^-v):
+ * the product rule on v * sigma(v) with sigma' = sigma (1 - sigma).  Used to
+ * carry the gate's error term through the SwiGLU epilogue. */
+static double silu_grad(double v)
+{
+    const double sig = 1.0 / (1.0 + exp(-v));
+    return sig * (1.0 + v * (1.0 - sig));
+}
+
 /* y = epilogue(x . W^T) in fp64 for all m < M and output columns n < Nout
  * (Nout = N/2 for SwiGLU, else N).  y and tol are [M, Nout] row-major;
  * tol gets the T term (for SwiGLU the propagated
@@ -460,14 +469,14 @@ EXPORT void mxr_gemm(const uint8_t *a, const void *sa, int a_fmt,
         dot_one(a, sa, a_fmt, b, sb, b_fmt, m, n, K, &acc, &aabs);
         if (epi == EPI_SWIGLU) {
             double g = acc + (bias ? (double)bias[n] : 0.0);
-            double u_acc, u_abs, u, sg, dsg, sig;
+            double u_acc, u_abs, u, sg, dsg;
             dot_one(a, sa, a_fmt, b, sb, b_fmt, m, n + Nout, K, &u_acc, &u_abs);
             u = u_acc + (bias ? (double)bias[n + Nout] : 0.0);
             sg = silu(g);
-            /* d/dg silu(g) = sigma(g) (1 + g (1 - sigma(g))) */
-            sig = 1.0 / (1.0 + exp(-g));
-            dsg = sig * (1.0 + g * (1.0 - sig));
+            dsg = silu_grad(g);
             out = sg * u;
+            /* first-order propagation of |d acc_g| <= T_g and |d acc_u| <= T_u
+             * through y = silu(g) u */
             t = fabs(dsg) * aabs * fabs(u) + fabs(sg) * u_abs;
         } else {
             double v = acc;
@@ -484,3 +493,4 @@ EXPORT void mxr_gemm(const uint8_t *a, const void *sa, int a_fmt,
 /* Exposed for the epilogue pins. */
 EXPORT double mxr_gelu_tanh(double v) { return gelu_tanh(v); }
 EXPORT double mxr_silu(double v) { return silu(v); }
+EXPORT double mxr_silu_grad(double v) { return silu_grad(v); }

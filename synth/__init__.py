@@ -72,6 +72,11 @@ def u64(seed: int, idx: torch.Tensor) -> torch.Tensor:
 def normal_f64(seed: int, start: int, count: int, device="cpu") -> torch.Tensor:
     """fp64 standard normals for stream elements [start, start + count)."""
     e = torch.arange(start, start + count, dtype=torch.int64, device=device)
+    return normal_f64_at(seed, e)
+
+
+def normal_f64_at(seed: int, e: torch.Tensor) -> torch.Tensor:
+    """fp64 standard normals for the stream elements listed in ``e`` (int64)."""
     r0 = u64(seed, 2 * e)
     r1 = u64(seed, 2 * e + 1)
     u1 = (_lsr(r0, 11) + 1).to(torch.float64) * 2.0 ** -53
@@ -96,11 +101,18 @@ def bf16_matrix(seed: int, rows: int, cols: int, sigma: float, row0: int = 0,
     return out.view(nrows, cols)
 
 
-def bf16_rows(seed: int, cols: int, sigma: float, row_ids, device="cpu") -> torch.Tensor:
+def bf16_rows(seed: int, cols: int, sigma: float, row_ids, device="cpu",
+              chunk: int = 1 << 24) -> torch.Tensor:
     """Selected rows (any order) of a seeded matrix with ``cols`` columns."""
-    parts = [bf16_matrix(seed, int(r) + 1, cols, sigma, row0=int(r), nrows=1,
-                         device=device) for r in row_ids]
-    return torch.cat(parts, 0) if parts else torch.empty(0, cols, dtype=torch.bfloat16)
+    ids = torch.as_tensor([int(r) for r in row_ids], dtype=torch.int64, device=device)
+    out = torch.empty(len(ids) * cols, dtype=torch.bfloat16, device=device)
+    per = max(1, chunk // cols)
+    col = torch.arange(cols, dtype=torch.int64, device=device)
+    for i in range(0, len(ids), per):
+        r = ids[i:i + per]
+        z = normal_f64_at(seed, (r[:, None] * cols + col[None, :]).reshape(-1)) * sigma
+        out[i * cols:(i + len(r)) * cols] = z.to(torch.float32).to(torch.bfloat16)
+    return out.view(len(ids), cols)
 
 
 def f32_vector(seed: int, n: int, sigma: float, device="cpu") -> torch.Tensor:

@@ -10,6 +10,7 @@ import synth
 
 EPI_NEEDS_BIAS = (1, 2)
 SENTINEL = 0x7FA5  # a bf16 NaN pattern no kernel writes
+WS_GUARD, WS_SENTINEL = 256, 0xA5  # workspace guard bands (256 bytes keep its alignment)
 
 
 def to_dev(a, dtype=None):
@@ -84,6 +85,11 @@ class Case:
                 wsb = mx.workspace(self.M, self.N, self.K, self.a_fmt, self.b_fmt, self.epi)
             else:
                 wsb = mx.workspace()
+            # the workspace sits between two 256-byte guard bands of a
+            # sentinel byte, checked untouched afterwards
+            ws_full = torch.full((wsb.numel() + 2 * WS_GUARD,), WS_SENTINEL, dtype=torch.uint8, device="cuda")
+            ws_full[WS_GUARD:WS_GUARD + wsb.numel()] = 0
+            wsb = ws_full[WS_GUARD:WS_GUARD + wsb.numel()]
             plan = mx.mx_gemm_plan_info(self.M, self.N, self.K, a_fmt, self.b_fmt, self.epi, wsb.numel())
             self.last_ws = wsb
             self.last_plan = plan
@@ -95,6 +101,9 @@ class Case:
         torch.cuda.synchronize()
         assert mx.mx_workspace_status(wsb) == 0, "a bounded wait ran out"
         assert guards_intact(full), "write outside the output"
+        wg = ws_full.cpu().numpy()
+        assert (wg[:WS_GUARD] == WS_SENTINEL).all() and (wg[-WS_GUARD:] == WS_SENTINEL).all(), \
+            "write outside the workspace"
         # everything after the 256-byte status block (arrival counters, and the
         # decode kernel's fp32 accumulators) is back to zero: the last arrival
         # of every tile reset its own
@@ -113,7 +122,7 @@ class Case:
             bad = np.argwhere(~ok)
             i, j = bad[0]
             err = np.abs(y_gpu - y)
-            bound = 2.0 ** -8 * np.abs(y) + 1e-5 * t
+            bound = oracle.tolerance_bound(y, t)
             worst = np.unravel_index(np.argmax(err / np.maximum(bound, 1e-300)), err.shape)
             raise AssertionError(
                 f"{what}: {len(bad)} of {ok.size} outside tolerance; first ({i},{j}) gpu={y_gpu[i, j]!r} "

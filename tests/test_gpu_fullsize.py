@@ -4,10 +4,12 @@ weight prefetch), checked against the fp64 oracle on sampled outputs.
 
 The oracle never sees a value produced on the GPU: it regenerates the sampled
 rows of x and W from the seeded generator, quantises them itself, and computes
-those outputs; the GPU quantises and multiplies the full matrices.  Sampled
-rows include the first and last token; sampled columns are whole 32-column
-blocks (so 32 x 32 weight scales are regenerated exactly) including the last
-one, and, for SwiGLU, the matching gate and up rows."""
+those outputs; the GPU quantises and multiplies the full matrices.  The samples
+follow the launch plan the library chose: at least one row inside every tile
+of rows (all rows for the decode kernels, whose one tile holds every token)
+and one whole 32-column block inside every tile of output columns, the ragged
+last tiles included; for SwiGLU the matching gate and up rows of W come with
+each block.  Whole 32-column blocks keep 32 x 32 weight scales regenerable."""
 import numpy as np
 import pytest
 import torch
@@ -33,13 +35,36 @@ WORKLOADS = [
 ]
 
 
-def sample_rows(M, rng, n=14):
-    rows = {0, M - 1, M // 2} | set(rng.integers(0, M, size=n).tolist())
+def plan_tiles(plan, M, swiglu):
+    """(rows per tile, output columns per tile) of the plan that ran."""
+    if plan["kernel"] == "decode":
+        # one tile of tokens; 128 weight rows (or 240 on the MMA's N side) per
+        # output tile, a gate and an up sub-tile of 128 each for SwiGLU
+        return M, (128 if plan["weights_on"] == "M" else (120 if swiglu else 240))
+    bn = plan["block_n"]
+    return plan["block_m"], (bn // 2 if swiglu else bn)
+
+
+def sample_rows(M, tile_m, rng):
+    """One random row inside every tile of rows, plus the first and last row."""
+    if tile_m >= M:
+        return np.arange(M, dtype=np.int64)
+    rows = {0, M - 1}
+    for r0 in range(0, M, tile_m):
+        rows.add(int(rng.integers(r0, min(r0 + tile_m, M))))
     return np.array(sorted(rows), np.int64)
 
 
-def sample_blocks(nblocks, rng, n=3):
-    blocks = {0, nblocks - 1, nblocks // 2} | set(rng.integers(0, nblocks, size=n).tolist())
+def sample_blocks(nout, tile_n, rng):
+    """One whole 32-column block inside every tile of output columns (the
+    block holding a tile's last column when no block fits inside it), plus the
+    first and last block."""
+    assert nout % 32 == 0
+    blocks = {0, nout // 32 - 1}
+    for c0 in range(0, nout, tile_n):
+        c1 = min(c0 + tile_n, nout)
+        first, last = -(-c0 // 32), c1 // 32 - 1  # blocks wholly inside [c0, c1)
+        blocks.add(int(rng.integers(first, last + 1)) if first <= last else (c1 - 1) // 32)
     return np.array(sorted(blocks), np.int64)
 
 
@@ -82,13 +107,19 @@ def test_full_size_sampled(mx, name, M, N, K, b_fmt, epi, seed, with_bias):
     del g
 
     # ---- oracle: sampled rows x sampled 32-column blocks, from its own quantisation
+    plan = mx.mx_gemm_plan_info(M, N, K, a_fmt, b_fmt, epi, wsb.numel())
+    tile_m, tile_n = plan_tiles(plan, M, epi == SWIGLU)
     rng = np.random.default_rng(seed * 7919 + M)
-    rows = sample_rows(M, rng)
+    rows = sample_rows(M, tile_m, rng)
     nout = N // 2 if epi == SWIGLU else N
-    cols = (sample_blocks(nout // 32, rng)[:, None] * 32 + np.arange(32)[None, :]).ravel()
+    blocks = sample_blocks(nout, tile_n, rng)
+    assert len(blocks) >= -(-nout // tile_n) and len(rows) >= min(M, -(-M // tile_m))
+    cols = (blocks[:, None] * 32 + np.arange(32)[None, :]).ravel()
     w_rows = np.concatenate([cols, cols + N // 2]) if epi == SWIGLU else cols
-    xs = synth.bf16_rows(seed, K, synth.X_SIGMA, rows)
-    wsel = synth.bf16_rows(seed + 1, K, synth.W_SIGMA, w_rows)
+    # the sampled rows are drawn on the device (the generator is counter based,
+    # so they are the rows the GPU multiplied) and handed to the oracle
+    xs = synth.bf16_rows(seed, K, synth.X_SIGMA, rows, device=dev).cpu()
+    wsel = synth.bf16_rows(seed + 1, K, synth.W_SIGMA, w_rows, device=dev).cpu()
     a_codes, a_scales = oracle.quant_act(xs, a_fmt)
     b_codes, b_scales = oracle.quant_weight(wsel, b_fmt)
     bsel = None

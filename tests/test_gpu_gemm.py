@@ -172,3 +172,35 @@ def test_two_row_block_tiles(mx, b_fmt, epi):
 def test_auto_plan_uses_two_row_blocks_for_large_m(mx):
     plan = mx.mx_gemm_plan(4096, 4096, 4096, 0, 0, 2)
     assert plan["block_n"] == 240 and plan["splits"] == 1
+
+
+@pytest.mark.parametrize("plan", ["tile", "decode", "split-ws", "split-cluster"])
+@pytest.mark.parametrize("b_fmt,epi", [(E2, SWIGLU), (E8, GELU), (F32, SWIGLU), (E8, SWIGLU)])
+def test_epilogue_far_tails(mx, plan, b_fmt, epi):
+    # biases spread over [-120, 120] push the gate / GELU pre-activations into
+    # the far tails, where e^-v leaves the fp32 range: SiLU(g) and GELU(v)
+    # there are tiny (down to bf16 subnormals), and must come out as such
+    M = 300 if plan == "tile" else 16
+    N, K = 512, 512
+    c = Case(M, N, K, a_fmt_for(b_fmt), b_fmt, epi, seed=70 + b_fmt * 10 + epi)
+    gen = torch.Generator().manual_seed(5)
+    if epi == SWIGLU:
+        gate = torch.linspace(-120.0, 120.0, N // 2)[torch.randperm(N // 2, generator=gen)]
+        up = torch.randn(N // 2, generator=gen) * 3
+        c.bias = torch.cat([gate, up]).float()
+    else:
+        c.bias = torch.linspace(-120.0, 120.0, N)[torch.randperm(N, generator=gen)].float()
+    c._ref = None
+    kw = {"tile": dict(decode=-1), "decode": dict(decode=1),
+          "split-ws": dict(decode=-1, block_n=128, splits=4),
+          "split-cluster": dict(decode=-1, block_n=128, splits=4, ws="min")}[plan]
+    y = c.run_gpu(mx, **kw)
+    yref, _ = c.ref()
+    if epi == SWIGLU:
+        # outputs far below fp32's e^-88 reach, down to bf16 subnormals (the
+        # fp64 tanh form of GELU is exactly 0 there, so GELU is checked for
+        # finite, in-tolerance tails only)
+        tiny = (np.abs(yref) < 2.0 ** -120) & (yref != 0)
+        assert tiny.any(), "the case does not reach the far tail"
+    assert np.isfinite(y).all()
+    c.check(y, f"tails {plan} fmt{b_fmt} epi{epi}")

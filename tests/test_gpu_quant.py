@@ -86,3 +86,32 @@ def test_quant_weight_e2m1_every_bf16_pattern(mx):
     torch.cuda.synchronize()
     assert np.array_equal(s.cpu().numpy(), scales)
     assert np.array_equal(c.cpu().numpy(), codes)
+
+
+@pytest.mark.parametrize("M,K", [(4096, 4096), (4096, 5120)])
+def test_quant_act_e8m0_bit_exact_prefill_sizes(mx, M, K):
+    # the DiT/ViT MLP and W4A8 gate_up prefill activations: several passes of
+    # the kernel's grid-stride loop over the blocks
+    x = synth.bf16_matrix(2 if K == 4096 else 3, M, K, synth.X_SIGMA, device="cuda")
+    x[M - 1, -32:] = 0
+    c, s = mx.act_buffers(M, K)
+    mx.mx_quant_act(x, c, s)
+    torch.cuda.synchronize()
+    codes, scales = oracle.quant_act_e8m0(x.cpu())
+    assert np.array_equal(s.cpu().numpy(), scales)
+    assert np.array_equal(c.cpu().numpy(), codes)
+
+
+@pytest.mark.parametrize("fmt,N,K", [(1, 34816, 5120), (0, 34816, 5120), (0, 4096, 4096)])
+def test_quant_weight_bit_exact_full_sizes(mx, fmt, N, K):
+    # the full gate_up weight as e2m1 and as e4m3 with 32 x 32 blocks (several
+    # grid-stride passes of either kernel), and the MLP weight
+    seed = 3 if N == 34816 else 2
+    w = synth.bf16_matrix(seed + 1, N, K, synth.W_SIGMA, device="cuda")
+    c, s = mx.weight_buffers(N, K, fmt)
+    mx.mx_quant_weight(w, c, s, fmt)
+    torch.cuda.synchronize()
+    codes, scales = oracle.quant_weight(w.cpu(), fmt)
+    del w
+    assert np.array_equal(s.cpu().numpy(), scales)
+    assert np.array_equal(c.cpu().numpy(), codes)

@@ -383,6 +383,160 @@ def test_swiglu_pairs_gate_rows_with_up_rows(oracle_mod):
     assert np.allclose(y0, F.silu(torch.from_numpy(acc[:, :64])).numpy() * acc[:, 64:], rtol=1e-13, atol=1e-16)
 
 
+# ---- the SwiGLU tolerance term ------------------------------------------------
+#
+# For SwiGLU the acceptance bound carries the GEMM's error terms through the
+# epilogue to first order: |d acc_g| <= 1e-5 T_g and |d acc_u| <= 1e-5 T_u move
+# y = silu(g) u by at most |silu'(g)| T_g |u| + |silu(g)| T_u (times 1e-5).
+# The checks below tie that term to autograd, to finite differences and to a
+# brute-force propagation on dequantised operands; the planted-mistake test
+# rebuilds the oracle with a wrong term and shows that they catch it.
+
+def _check_silu_grad(om):
+    v = np.concatenate([np.linspace(-30, 30, 1201), [0.0, 1e-8, -1e-8, 5.0, -5.0]])
+    got = np.array([om.silu_grad(x) for x in v])
+    tv = torch.from_numpy(v).requires_grad_(True)
+    F.silu(tv).sum().backward()
+    assert np.allclose(got, tv.grad.numpy(), rtol=1e-12, atol=1e-15), "silu' differs from autograd"
+    h = 1e-5
+    fd = np.array([(om.silu(x + h) - om.silu(x - h)) / (2 * h) for x in v])
+    assert np.allclose(got, fd, rtol=1e-7, atol=1e-9), "silu' differs from the central difference"
+    assert om.silu_grad(0.0) == 0.5  # sigma(0) (1 + 0) = 1/2
+
+
+def _dequant_swiglu(om, seed, M, N, K, b_fmt):
+    a, sa, bc, sb, bias = _problem(om, seed, M, N, K, 0, b_fmt)
+    A = _dequant_a(a, sa, 0, K)
+    B = _dequant_b(bc, sb, b_fmt, N, K, om)
+    return a, sa, bc, sb, bias, A, B
+
+
+def _check_swiglu_term(om, b_fmt):
+    M, N, K = 4, 128, 96
+    a, sa, bc, sb, bias, A, B = _dequant_swiglu(om, 15 + b_fmt, M, N, K, b_fmt)
+    y, t = om.gemm(a, sa, 0, bc, sb, b_fmt, bias, 3, M, N, K)
+    h = N // 2
+    bb = bias.double().numpy()
+    g = A @ B[:h].T + bb[None, :h]
+    u = A @ B[h:].T + bb[None, h:]
+    t_g = np.abs(A) @ np.abs(B[:h]).T
+    t_u = np.abs(A) @ np.abs(B[h:]).T
+    gt = torch.from_numpy(g).requires_grad_(True)
+    s = F.silu(gt)
+    s.sum().backward()
+    want = np.abs(gt.grad.numpy()) * t_g * np.abs(u) + np.abs(s.detach().numpy()) * t_u
+    assert np.allclose(t, want, rtol=1e-12, atol=0), "SwiGLU T differs from the brute-force propagation"
+
+
+def _check_swiglu_term_is_tight(om):
+    # One token.  Perturbing every gate product a_k w_gk by eps |a_k w_gk| with
+    # the sign of silu'(g) u moves y by eps |silu'(g)| T_g |u| to first order;
+    # the up products, likewise, by eps |silu(g)| T_u.  The two perturbations
+    # together reach eps T, and random signs stay inside it.
+    M, N, K = 1, 128, 96
+    a, sa, bc, sb, bias, A, B = _dequant_swiglu(om, 19, M, N, K, 1)
+    y, t = om.gemm(a, sa, 0, bc, sb, 1, bias, 3, M, N, K)
+    h = N // 2
+    bb = bias.double().numpy()
+
+    def swiglu(Bm):
+        g = torch.from_numpy(A @ Bm[:h].T + bb[None, :h])
+        return (F.silu(g) * torch.from_numpy(A @ Bm[h:].T + bb[None, h:])).numpy()
+
+    y0 = swiglu(B)
+    g0 = A @ B[:h].T + bb[None, :h]
+    u0 = A @ B[h:].T + bb[None, h:]
+    gt = torch.from_numpy(g0).requires_grad_(True)
+    F.silu(gt).sum().backward()
+    dg = gt.grad.numpy()[0]
+    sg = F.silu(torch.from_numpy(g0)).numpy()[0]
+    eps = 1e-7
+    # w_nk += eps s sign(a_k) |w_nk| changes a_k w_nk by eps s |a_k w_nk|
+    a_sign = np.sign(A[0])[None, :]
+    s_gate = np.sign(dg * u0[0])[:, None]
+    s_up = np.sign(sg)[:, None]
+    Bp = B.copy()
+    Bp[:h] += eps * s_gate * a_sign * np.abs(B[:h])
+    Bp[h:] += eps * s_up * a_sign * np.abs(B[h:])
+    dy = (swiglu(Bp) - y0)[0]
+    assert np.allclose(dy, eps * t[0], rtol=1e-4, atol=0), "T is not the first-order bound it should be"
+    rng = np.random.default_rng(7)
+    for _ in range(3):
+        Br = B * (1 + eps * rng.uniform(-1, 1, B.shape))
+        assert (np.abs(swiglu(Br) - y0)[0] <= eps * t[0] * (1 + 1e-4)).all()
+
+
+def test_silu_grad_against_autograd_and_finite_differences(oracle_mod):
+    _check_silu_grad(oracle_mod)
+
+
+@pytest.mark.parametrize("b_fmt", [0, 1])
+def test_swiglu_tolerance_term_against_brute_force(oracle_mod, b_fmt):
+    _check_swiglu_term(oracle_mod, b_fmt)
+
+
+def test_swiglu_tolerance_term_is_the_tight_first_order_bound(oracle_mod):
+    _check_swiglu_term_is_tight(oracle_mod)
+
+
+# Mistakes planted in a rebuilt copy of the oracle (never in the oracle the
+# other tests use): each must make at least two of the checks above fail.
+SWIGLU_TERM_MUTANTS = [
+    ("sign flip inside the SiLU derivative",
+     "return sig * (1.0 + v * (1.0 - sig));", "return sig * (1.0 - v * (1.0 - sig));"),
+    ("|u| dropped from the gate term",
+     "t = fabs(dsg) * aabs * fabs(u) + fabs(sg) * u_abs;", "t = fabs(dsg) * aabs + fabs(sg) * u_abs;"),
+    ("gate and up error terms swapped",
+     "t = fabs(dsg) * aabs * fabs(u) + fabs(sg) * u_abs;", "t = fabs(dsg) * u_abs * fabs(u) + fabs(sg) * aabs;"),
+    ("derivative taken as sigma(g)",
+     "return sig * (1.0 + v * (1.0 - sig));", "return sig;"),
+]
+
+
+@pytest.mark.parametrize("what,old,new", SWIGLU_TERM_MUTANTS, ids=[m[0] for m in SWIGLU_TERM_MUTANTS])
+def test_swiglu_term_checks_catch_planted_mistakes(oracle_mod, tmp_path, what, old, new):
+    import subprocess
+    src_path = os.path.join(os.path.dirname(oracle_mod.__file__), "mxref.c")
+    src = open(src_path).read()
+    assert src.count(old) == 1, f"mutation site for '{what}' not found"
+    (tmp_path / "mxref.c").write_text(src.replace(old, new))
+    so = tmp_path / "_mxref_mutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-D_DEFAULT_SOURCE", "-fPIC", "-fopenmp", "-fno-fast-math",
+                    "-ffp-contract=off", "-shared", "-o", str(so), str(tmp_path / "mxref.c"), "-lm"], check=True)
+    mutant = oracle_mod.load_library(str(so))
+    saved = oracle_mod._LIB
+    caught = []
+    try:
+        oracle_mod._LIB = mutant
+        for name, check in [("silu_grad", lambda: _check_silu_grad(oracle_mod)),
+                            ("term e4m3", lambda: _check_swiglu_term(oracle_mod, 0)),
+                            ("term e2m1", lambda: _check_swiglu_term(oracle_mod, 1)),
+                            ("tight", lambda: _check_swiglu_term_is_tight(oracle_mod))]:
+            try:
+                check()
+            except AssertionError:
+                caught.append(name)
+    finally:
+        oracle_mod._LIB = saved
+    assert len(caught) >= 2, f"planted mistake '{what}' caught only by {caught}"
+
+
+def test_tolerance_accepts_correct_bf16_roundings_and_no_more(oracle_mod):
+    # The bound's first term stands for the bf16 rounding of the output: every
+    # correct rounding (torch's cast) of values across bf16's whole range,
+    # subnormals included, passes with T = 0; two bf16 steps away fails.
+    rng = np.random.default_rng(3)
+    n = 20000
+    y = np.where(rng.random(n) < 0.5, -1.0, 1.0) * np.exp2(rng.uniform(-140.0, 120.0, n))
+    yb = torch.from_numpy(y).to(torch.bfloat16)
+    t0 = np.zeros(n)
+    assert oracle_mod.within_tolerance(yb.double().numpy(), y, t0).all()
+    bits = yb.view(torch.int16).numpy().astype(np.int32)
+    far = torch.from_numpy((bits + 2).astype(np.int16)).view(torch.bfloat16).double().numpy()
+    normal = np.abs(y) >= 2.0 ** -124
+    assert not oracle_mod.within_tolerance(far, y, t0)[normal].any()
+
+
 def test_page_shapes_fixture(oracle_mod):
     # tests/golden/page_shapes.txt: layouts the pages print.
     path = os.path.join(GOLDEN, "page_shapes.txt")
