@@ -207,7 +207,10 @@ class Workload:
         copies = min(64, max(1, math.ceil(2 * L2_BYTES / self.w_bytes)))
         self.weights = [(wc, ws)] + [(wc.clone(), ws.clone()) for _ in range(copies - 1)]
         self.bias = synth.f32_vector(seed + 2, N, synth.BIAS_SIGMA, device=dev) if with_bias else None
-        self.nout = N // 2 if epi == mx.MX_EPI_SWIGLU else N
+        self.nout = N // 2 if epi in (mx.MX_EPI_SWIGLU, mx.MX_EPI_SWIGLU_MXQ) else N
+        # bytes of one output row: bf16, or e4m3 codes + E8M0 scales when the
+        # SwiGLU output is handed on as the next GEMM's MX operand
+        self.out_row_bytes = (N // 2 + N // 64) if epi == mx.MX_EPI_SWIGLU_MXQ else 2 * self.nout
         self.x, self.acodes, self.ascales, self.out = {}, {}, {}, {}
         for M in self.Ms:
             self.x[M] = synth.bf16_matrix(seed, M, K, synth.X_SIGMA, device=dev)
@@ -225,20 +228,24 @@ class Workload:
     def flops(self, M):
         return 2.0 * M * self.N * self.K
 
+    def act_bytes(self, M):
+        """Activation codes + scales of M rows."""
+        if self.a_fmt == 3:  # packed e2m1 + 1x32 E8M0
+            return M * self.K // 2 + M * (self.K // 32)
+        return M * self.K + (M * (self.K // 32) if self.a_fmt == 0 else 4 * M)
+
     def gemm_bytes(self, M):
         """Algorithmic bytes of one GEMM launch: weights + their scales, activation
-        codes + scales, and the bf16 output."""
-        a_sc = M * (self.K // 32) if self.a_fmt == 0 else 4 * M
-        return self.w_bytes + M * self.K + a_sc + 2 * M * self.nout
+        codes + scales, and the output."""
+        return self.w_bytes + self.act_bytes(M) + M * self.out_row_bytes
 
     def fused_bytes(self, M):
         """Algorithmic bytes of one fused launch: weights + their scales, the bf16
-        activations, and the bf16 output."""
-        return self.w_bytes + 2 * M * self.K + 2 * M * self.nout
+        activations, and the output."""
+        return self.w_bytes + 2 * M * self.K + M * self.out_row_bytes
 
     def quant_bytes(self, M):
-        sc = M * (self.K // 32) if self.a_fmt == 0 else 4 * M
-        return 2 * M * self.K + M * self.K + sc
+        return 2 * M * self.K + self.act_bytes(M)
 
     def next_weights(self):
         wc, ws = self.weights[self.rot % len(self.weights)]
@@ -430,6 +437,12 @@ def roofline_entry(wl: Workload, M, t_gemm, pk, bound, fused=False):
                 "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
                 "peak_note": f"{pk['source']} HBM copy bandwidth"}
     ach = wl.flops(M) / t_gemm / 1e12
+    if wl.a_fmt == 3:
+        # W4A4 runs at the fp4 rate: 4x bf16 (nominal ratio 9 / 2.25)
+        fp4_peak = 4.0 * pk["bf16_tflops"]
+        return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                "frac": round(ach / fp4_peak, 4), "traffic": None,
+                "peak_note": f"fp4 = 4 x {pk['source']} bf16 burst", "frac_of_spec_9000": round(ach / 9000.0, 4)}
     fp8_peak = 2.0 * pk["bf16_tflops"]  # dense fp8 = 2x bf16 (nominal ratio 4.5 / 2.25)
     return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
             "frac": round(ach / fp8_peak, 4), "traffic": None,
@@ -785,6 +798,15 @@ PROFILE_SPECS = {
     "gateup4096": ((4096,), 34816, 5120, 0, 1, 3, 3, False, "tensor",
                    "W4A8 gate_up + SwiGLU, prefill (M4096 N34816 K5120)"),
     "lmhead": ((16,), 248320, 5120, 1, 2, 0, 4, False, "hbm", "fp8 per-channel lm_head (M16 N248320 K5120)"),
+    # the same FFN's neighbours: the gate_up handing its SwiGLU output on as MX
+    # codes, the down projection that takes them, and the gate_up as W4A4
+    "gateup16_mxq": ((16,), 34816, 5120, 0, 1, 5, 3, False, "hbm",
+                     "W4A8 gate_up + SwiGLU -> e4m3 + 1x32 E8M0 codes, decode (M16 N34816 K5120)"),
+    "down16": ((16,), 5120, 17408, 0, 1, 0, 5, False, "hbm", "W4A8 down projection, decode (M16 N5120 K17408)"),
+    "down4096": ((4096,), 5120, 17408, 0, 1, 0, 5, False, "tensor",
+                 "W4A8 down projection, prefill (M4096 N5120 K17408)"),
+    "gateup4096_w4a4": ((4096,), 34816, 5120, 3, 1, 3, 3, False, "tensor",
+                        "W4A4 gate_up + SwiGLU, prefill (M4096 N34816 K5120), kind::mxf4"),
 }
 
 
@@ -816,7 +838,8 @@ def extra_workloads(mx, stream, pk):
     """The other workloads, each GEMM timed alone (graph of back-to-back
     launches over rotating weights) against its roofline."""
     res = []
-    for key in ("small", "mlp", "gateup16", "gateup4096", "lmhead"):
+    for key in ("small", "mlp", "gateup16", "gateup4096", "lmhead", "gateup16_mxq", "down16", "down4096",
+                "gateup4096_w4a4"):
         Ms, N, K, af, bf, epi, seed, bias, bound, name = PROFILE_SPECS[key]
         log(f"workload: {name}")
         try:

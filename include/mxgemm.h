@@ -81,7 +81,16 @@ typedef enum mx_a_fmt {
      * minimum, or mx_gemm_noalloc -- the decode kernel quantises them itself
      * in the same launch.  Pairs with the E8M0 weight formats.  Not an output
      * format of mx_quant_act. */
-    MX_A_BF16_E8M0_1X32 = 2
+    MX_A_BF16_E8M0_1X32 = 2,
+    /* W4A4: e2m1 codes packed two per byte [M, K/2] (low nibble = even k) +
+     * uint8 E8M0 scales [M, K/32], k the smallest integer with
+     * amax <= 6 * 2^k (the rule of the e2m1 weights), codes RNE onto the e2m1
+     * grid.  Pairs with MX_B_E2M1_E8M0_1X32 only (the native MXFP4 W4A4 GEMM,
+     * the sly-radiance README's AITER gemm_afp4wfp4 path) and runs at the
+     * tensor cores' fp4 rate (tcgen05.mma kind::mxf4, K = 64 per
+     * instruction); M > 64 and M <= 64 both take the tile kernel, no K split.
+     * mx_quant_act produces it from bf16. */
+    MX_A_E2M1_E8M0_1X32 = 3
 } mx_a_fmt;
 
 /* Weight operand formats (B = W, stored [N, K]). */
@@ -101,11 +110,25 @@ typedef enum mx_epi {
     MX_EPI_BIAS = 1,           /* y = acc + bias[n]                               */
     MX_EPI_BIAS_GELU_TANH = 2, /* v = acc + bias[n]; y = 0.5 v (1 + tanh(
                                   sqrt(2/pi) (v + 0.044715 v^3)))                */
-    MX_EPI_SWIGLU = 3          /* W = [gate; up] with N rows (gate rows 0..N/2-1,
+    MX_EPI_SWIGLU = 3,         /* W = [gate; up] with N rows (gate rows 0..N/2-1,
                                   up rows N/2..N-1); out [M, N/2]:
                                   y[m, j] = silu(g) * u, g = acc[m, j] (+ bias[j]),
                                   u = acc[m, j + N/2] (+ bias[j + N/2]),
                                   silu(v) = v / (1 + e^-v)                        */
+    MX_EPI_RESIDUAL = 4,       /* in place: out[m, n] = out[m, n] + (acc + bias[n]),
+                                  bias optional, computed in fp32 and rounded once
+                                  to bf16: the residual update x += y + b of the
+                                  ViT page's `vt_add`.  out holds the residual
+                                  stream on entry and must not overlap the
+                                  activations or weights                          */
+    MX_EPI_SWIGLU_MXQ = 5      /* MX_EPI_SWIGLU with its result handed on as the
+                                  next GEMM's MX operand (the sly README's fused
+                                  silu_mul_quant): y = bf16(silu(g) * u) is not
+                                  stored; out receives its 1 x 32 E8M0
+                                  quantisation, e4m3 codes [M, N/2] followed by
+                                  E8M0 scales [M, N/64] from byte M * N/2 of
+                                  out -- bit for bit what mx_quant_act gives for
+                                  that y, ready for MX_A_E4M3_E8M0_1X32         */
 } mx_epi;
 
 /*
@@ -122,6 +145,10 @@ typedef enum mx_epi {
  *           saturating), the sign of zero kept.
  *           MX_A_E4M3_F32_ROW: [M] fp32 -- s = amax_row / 448 (IEEE division;
  *           1.0 for an all-zero row); codes = RNE_satfinite(x / s).
+ *           MX_A_E2M1_E8M0_1X32: codes [M, K/2] packed e2m1 (low nibble =
+ *           even k), scales [M, K/32] E8M0 with k the smallest integer such
+ *           that amax <= 6 * 2^k; codes RNE onto {0, .5, 1, 1.5, 2, 3, 4, 6}
+ *           of x * 2^-k, the sign kept.
  *   Requires M >= 1, K >= 32, K % 32 == 0.  The result is bit-exact: it is the
  *   unique rounding the definition gives.
  */
@@ -143,6 +170,34 @@ MX_API mx_status mx_quant_act(const void* x, int M, int K, void* codes, void* sc
  *   MX_B_E4M3_F32_ROW: codes [N, K] uint8, scales [N] fp32 = amax_row / 448.
  */
 MX_API mx_status mx_quant_weight(const void* w, int N, int K, void* codes, void* scales, mx_b_fmt fmt, void* stream);
+
+/*
+ * mx_add_rms_quant -- residual add, RMSNorm and 1 x 32 E8M0 quantisation of
+ * each row: the producer that hands the next GEMM its MX operand (sly-radiance
+ * README, Contents table, radiance_fused_norm.py row: the fused add_rms_quant
+ * op returns (q_fp8, scale) for the W4A8 linear; RMSNorm with a plain weight as
+ * the DiT page's `rms_norm` defines it, x * rsqrt(mean x^2 + eps) * w).  Read
+ * as the unfused chain it replaces, for each row m:
+ *   r = bf16(x + residual), written back into `residual` (in place);
+ *   y = bf16(r * rsqrt(mean_k r^2 + eps) * w);
+ *   codes + scales = the 1 x 32 E8M0 quantisation of y, bit for bit what
+ *   mx_quant_act gives for that y; y itself goes to y_out when it is not NULL.
+ *
+ *   x         [M, K] bf16, device, read.
+ *   residual  [M, K] bf16, device, read and overwritten with r (may be x).
+ *   w         [K] bf16, device, read.
+ *   eps       >= 0.
+ *   y_out     [M, K] bf16, device, written; NULL = not wanted.
+ *   codes     [M, K] uint8 e4m3, device, written.
+ *   scales    [M, K/32] uint8 E8M0, device, written.
+ * The sum of squares is taken in fp32, so y can differ from an fp64 chain by
+ * one bf16 rounding where it falls near a bf16 midpoint; codes and scales are
+ * always those of the y written.  Requires M >= 1, 32 <= K <= 16384,
+ * K % 32 == 0; x, residual, w, codes and y_out 16-byte aligned.  Errors as
+ * mx_quant_act; no workspace.
+ */
+MX_API mx_status mx_add_rms_quant(const void* x, void* residual, const void* w, float eps, int M, int K,
+                                  void* y_out, void* codes, void* scales, void* stream);
 
 /*
  * mx_gemm_workspace_size -- bytes of workspace that let mx_gemm run its fastest

@@ -17,9 +17,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmxgemm.so")
 
 # formats and epilogues (values of the C enums)
-MX_A_E4M3_E8M0_1X32, MX_A_E4M3_F32_ROW, MX_A_BF16_E8M0_1X32 = 0, 1, 2
+MX_A_E4M3_E8M0_1X32, MX_A_E4M3_F32_ROW, MX_A_BF16_E8M0_1X32, MX_A_E2M1_E8M0_1X32 = 0, 1, 2, 3
 MX_B_E4M3_E8M0_32X32, MX_B_E2M1_E8M0_1X32, MX_B_E4M3_F32_ROW = 0, 1, 2
-MX_EPI_NONE, MX_EPI_BIAS, MX_EPI_BIAS_GELU_TANH, MX_EPI_SWIGLU = 0, 1, 2, 3
+MX_EPI_NONE, MX_EPI_BIAS, MX_EPI_BIAS_GELU_TANH, MX_EPI_SWIGLU, MX_EPI_RESIDUAL = 0, 1, 2, 3, 4
+MX_EPI_SWIGLU_MXQ = 5
 
 MX_LAUNCH_PDL, MX_LAUNCH_PREFETCH_WEIGHTS, MX_LAUNCH_DETERMINISTIC = 1, 2, 4
 MX_TUNE_BM_PAIR = 2  # mx_set_tuning block_m: 256 x 240 tiles over CTA pairs
@@ -27,7 +28,7 @@ MX_TUNE_BM_PAIR = 2  # mx_set_tuning block_m: 256 x 240 tiles over CTA pairs
 MX_OK, MX_ERR_NULL, MX_ERR_SHAPE, MX_ERR_ALIGN, MX_ERR_FORMAT = 0, 1, 2, 3, 4
 MX_ERR_WORKSPACE, MX_ERR_ARCH, MX_ERR_CUDA, MX_ERR_TIMEOUT = 5, 6, 7, 8
 
-EXPORTS = ["mx_quant_act", "mx_quant_weight", "mx_gemm_workspace_size", "mx_gemm", "mx_status_string",
+EXPORTS = ["mx_quant_act", "mx_quant_weight", "mx_add_rms_quant", "mx_gemm_workspace_size", "mx_gemm", "mx_status_string",
            "mx_workspace_status", "mx_debug_watchdog", "mx_set_tuning", "mx_gemm_plan", "mx_gemm_noalloc",
            "mx_debug_set_timeline", "mx_set_launch_flags", "mx_set_decode_tuning", "mx_gemm_plan_info"]
 
@@ -65,6 +66,7 @@ def load(path: str | None = None):
     sig = {
         "mx_quant_act": (I, [P, I, I, P, P, I, P]),
         "mx_quant_weight": (I, [P, I, I, P, P, I, P]),
+        "mx_add_rms_quant": (I, [P, P, P, ctypes.c_float, I, I, P, P, P, P]),
         "mx_gemm_workspace_size": (S, [I, I, I, I, I, I]),
         "mx_gemm": (I, [P, P, I, P, P, I, P, I, P, I, I, I, P, S, P]),
         "mx_status_string": (ctypes.c_char_p, [I]),
@@ -125,6 +127,14 @@ def mx_quant_weight(w, codes, scales, fmt, stream=None):
     """w bf16 [N, K] -> weight codes and scales in the chosen B format."""
     N, K = w.shape
     _check(load().mx_quant_weight(_p(w), N, K, _p(codes), _p(scales), fmt, _stream(stream)), "mx_quant_weight")
+
+
+def mx_add_rms_quant(x, residual, w, eps, y_out, codes, scales, stream=None):
+    """residual <- bf16(x + residual); y = bf16(RMSNorm(residual) * w) into
+    y_out (None = not wanted); codes / scales = its 1 x 32 E8M0 quantisation."""
+    M, K = x.shape
+    _check(load().mx_add_rms_quant(_p(x), _p(residual), _p(w), float(eps), M, K, _p(y_out), _p(codes), _p(scales),
+                                   _stream(stream)), "mx_add_rms_quant")
 
 
 def mx_gemm_workspace_size(M, N, K, a_fmt, b_fmt, epi) -> int:
@@ -215,6 +225,9 @@ def mx_gemm_plan(M, N, K, a_fmt, b_fmt, epi):
 # ---- allocation helpers (torch is the allocator) ---------------------------------
 
 def act_buffers(M, K, fmt=MX_A_E4M3_E8M0_1X32, device="cuda"):
+    if fmt == MX_A_E2M1_E8M0_1X32:
+        return (torch.empty(M, K // 2, dtype=torch.uint8, device=device),
+                torch.empty(M, K // 32, dtype=torch.uint8, device=device))
     codes = torch.empty(M, K, dtype=torch.uint8, device=device)
     if fmt == MX_A_E4M3_E8M0_1X32:
         scales = torch.empty(M, K // 32, dtype=torch.uint8, device=device)
@@ -244,4 +257,15 @@ def workspace(M=1, N=1, K=32, a_fmt=0, b_fmt=0, epi=0, device="cuda", problems=(
 
 
 def out_buffer(M, N, epi, device="cuda"):
+    """The output of mx_gemm: bf16 [M, N] ([M, N/2] for SwiGLU); for
+    MX_EPI_SWIGLU_MXQ the bytes of e4m3 codes [M, N/2] and E8M0 scales
+    [M, N/64] (split it with mxq_views)."""
+    if epi == MX_EPI_SWIGLU_MXQ:
+        return torch.empty(M * (N // 2) + M * (N // 64), dtype=torch.uint8, device=device)
     return torch.empty(M, N // 2 if epi == MX_EPI_SWIGLU else N, dtype=torch.bfloat16, device=device)
+
+
+def mxq_views(out, M, N):
+    """(codes [M, N/2], scales [M, N/64]) views of an MX_EPI_SWIGLU_MXQ output."""
+    nc = M * (N // 2)
+    return out[:nc].view(M, N // 2), out[nc:nc + M * (N // 64)].view(M, N // 64)

@@ -56,18 +56,20 @@ mx_status validate_gemm(const void* a_codes, const void* a_scales, mx_a_fmt a_fm
 {
     const bool a_bf16 = a_fmt == MX_A_BF16_E8M0_1X32;  // a_scales unused
     if (!a_codes || (!a_scales && !a_bf16) || !b_codes || !b_scales || !out) return MX_ERR_NULL;
-    if (epi != MX_EPI_NONE && epi != MX_EPI_BIAS && epi != MX_EPI_BIAS_GELU_TANH && epi != MX_EPI_SWIGLU)
+    if (epi != MX_EPI_NONE && epi != MX_EPI_BIAS && epi != MX_EPI_BIAS_GELU_TANH && epi != MX_EPI_SWIGLU &&
+        epi != MX_EPI_RESIDUAL && epi != MX_EPI_SWIGLU_MXQ)
         return MX_ERR_FORMAT;
     const bool pair_ok = ((a_fmt == MX_A_E4M3_E8M0_1X32 || a_bf16) &&
                           (b_fmt == MX_B_E4M3_E8M0_32X32 || b_fmt == MX_B_E2M1_E8M0_1X32)) ||
-                         (a_fmt == MX_A_E4M3_F32_ROW && b_fmt == MX_B_E4M3_F32_ROW);
+                         (a_fmt == MX_A_E4M3_F32_ROW && b_fmt == MX_B_E4M3_F32_ROW) ||
+                         (a_fmt == MX_A_E2M1_E8M0_1X32 && b_fmt == MX_B_E2M1_E8M0_1X32);
     if (!pair_ok) return MX_ERR_FORMAT;
     if ((epi == MX_EPI_BIAS || epi == MX_EPI_BIAS_GELU_TANH) && !bias) return MX_ERR_NULL;
     if (epi == MX_EPI_NONE && bias) return MX_ERR_FORMAT;
     if (M < 1 || N < 1 || K < 32 || (K % 32) != 0) return MX_ERR_SHAPE;
     if (b_fmt == MX_B_E4M3_E8M0_32X32 && (N % 32) != 0) return MX_ERR_SHAPE;
     if (b_fmt == MX_B_E2M1_E8M0_1X32 && (K % 128) != 0) return MX_ERR_SHAPE;
-    if (epi == MX_EPI_SWIGLU && (N % 64) != 0) return MX_ERR_SHAPE;
+    if (epi_swiglu(epi) && (N % 64) != 0) return MX_ERR_SHAPE;
     if (!aligned(a_codes, 16) || !aligned(b_codes, b_fmt == MX_B_E2M1_E8M0_1X32 ? 32 : 16) || !aligned(out, 16))
         return MX_ERR_ALIGN;
     const uintptr_t sal = (a_fmt == MX_A_E4M3_F32_ROW) ? 4 : 1;
@@ -101,7 +103,7 @@ const char* mx_status_string(mx_status s)
 mx_status mx_quant_act(const void* x, int M, int K, void* codes, void* scales, mx_a_fmt fmt, void* stream)
 {
     if (!x || !codes || !scales) return MX_ERR_NULL;
-    if (fmt != MX_A_E4M3_E8M0_1X32 && fmt != MX_A_E4M3_F32_ROW) return MX_ERR_FORMAT;
+    if (fmt != MX_A_E4M3_E8M0_1X32 && fmt != MX_A_E4M3_F32_ROW && fmt != MX_A_E2M1_E8M0_1X32) return MX_ERR_FORMAT;
     if (M < 1 || K < 32 || (K % 32) != 0) return MX_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, fmt == MX_A_E4M3_F32_ROW ? 4 : 1))
         return MX_ERR_ALIGN;
@@ -111,7 +113,24 @@ mx_status mx_quant_act(const void* x, int M, int K, void* codes, void* scales, m
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (fmt == MX_A_E4M3_E8M0_1X32)
         return from_cuda(launch_quant_e8m0_1x32(x, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales), st));
+    if (fmt == MX_A_E2M1_E8M0_1X32)  // the 1 x 32 e2m1 rule of the weights, on rows of activations
+        return from_cuda(launch_quant_w_e2m1_1x32(x, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales), st));
     return from_cuda(launch_quant_f32_row(x, M, K, static_cast<uint8_t*>(codes), static_cast<float*>(scales), st));
+}
+
+mx_status mx_add_rms_quant(const void* x, void* residual, const void* w, float eps, int M, int K, void* y_out,
+                           void* codes, void* scales, void* stream)
+{
+    if (!x || !residual || !w || !codes || !scales) return MX_ERR_NULL;
+    if (M < 1 || K < 32 || (K % 32) != 0 || K > 16384 || !(eps >= 0.f)) return MX_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(residual, 16) || !aligned(w, 16) || !aligned(codes, 16) ||
+        (y_out && !aligned(y_out, 16)))
+        return MX_ERR_ALIGN;
+    DeviceInfo dev;
+    mx_status s = arch_ok(&dev);
+    if (s != MX_OK) return s;
+    return from_cuda(launch_add_rms_quant(x, residual, w, eps, M, K, y_out, codes, scales,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 mx_status mx_quant_weight(const void* w, int N, int K, void* codes, void* scales, mx_b_fmt fmt, void* stream)

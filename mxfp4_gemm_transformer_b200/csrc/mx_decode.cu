@@ -510,7 +510,20 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
                     tmem_ld16(abase + c, gv);
                     if (SWIGLU) tmem_ld16(abase + C::SUB_COLS + c, uv);
                     tmem_ld_wait();
-                    if (col_ok) {
+                    if (SWIGLU && p.q_codes) {
+                        // output handed on as MX codes: every lane takes part
+                        // (one 1 x 32 block per token per warp)
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) {
+                            const int m = c + t;  // the same token in every lane
+                            if (m < M) {
+                                const float sx = (SCALED || !col_ok) ? 1.f : __ldg(p.sxf + m);
+                                const float v = dec_epi<SWIGLU, !SCALED>(p.epi, __uint_as_float(gv[t]),
+                                                                         __uint_as_float(uv[t]), sx, bg, bu, wg, wu);
+                                dec_store_mxq(p, m, j, col_ok, lane, v);
+                            }
+                        }
+                    } else if (col_ok) {
 #pragma unroll
                         for (int t = 0; t < 16; ++t) {
                             const int m = c + t;
@@ -519,7 +532,7 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
                                 const float v = dec_epi<SWIGLU, !SCALED>(p.epi, __uint_as_float(gv[t]),
                                                                          SWIGLU ? __uint_as_float(uv[t]) : 0.f, sx, bg,
                                                                          bu, wg, wu);
-                                ocol[static_cast<size_t>(m) * p.Nout] = __float2bfloat16_rn(v);
+                                store_out(ocol + static_cast<size_t>(m) * p.Nout, p.epi, v);
                             }
                         }
                     }
@@ -581,11 +594,15 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
                             if (m < M) {
                                 __stcg(red + static_cast<size_t>(m) * 128, 0.f);
                                 if (SWIGLU) __stcg(red + static_cast<size_t>(M + m) * 128, 0.f);
-                                if (col_ok) {
+                                if (SWIGLU && p.q_codes) {
+                                    const float sx = (SCALED || !col_ok) ? 1.f : __ldg(p.sxf + m);
+                                    dec_store_mxq(p, m, j, col_ok, lane,
+                                                  dec_epi<SWIGLU, !SCALED>(p.epi, gv[t], uv[t], sx, bg, bu, wg, wu));
+                                } else if (col_ok) {
                                     const float sx = SCALED ? 1.f : __ldg(p.sxf + m);
                                     const float v = dec_epi<SWIGLU, !SCALED>(p.epi, gv[t], SWIGLU ? uv[t] : 0.f, sx,
                                                                              bg, bu, wg, wu);
-                                    ocol[static_cast<size_t>(m) * p.Nout] = __float2bfloat16_rn(v);
+                                    store_out(ocol + static_cast<size_t>(m) * p.Nout, p.epi, v);
                                 }
                             }
                         }
@@ -620,11 +637,44 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
             const int row_lo = crank * 128 / S, nrows = (crank + 1) * 128 / S - row_lo;
             const int M = p.M;
             const uint32_t part_s = smem_u32(wring);
+            if (SWIGLU && p.q_codes) {
+                // output handed on as MX codes: rank r finishes whole 32-row
+                // blocks b = r, r + S, ... of the tile's four (one 1 x 32
+                // quantisation block per token), one warp per token at a time
+                const int wid = static_cast<int>(threadIdx.x >> 5);
+                for (int b = crank; b < 4; b += S) {
+                    const int row = b * 32 + lane;
+                    const int j = tile * 128 + row;
+                    const bool col_ok = j < p.Nout;
+                    float bgv = 0.f, buv = 0.f, wgv = 1.f, wuv = 1.f;
+                    if (col_ok) {
+                        if (p.bias) {
+                            bgv = __ldg(p.bias + j);
+                            buv = __ldg(p.bias + j + p.n_half);
+                        }
+                        if (!SCALED) {
+                            wgv = __ldg(p.swf + j);
+                            wuv = __ldg(p.swf + j + p.n_half);
+                        }
+                    }
+                    for (int m = wid; m < M; m += kDecThreads / 32) {
+                        float sg = 0.f, su = 0.f;
+                        for (int q = 0; q < S; ++q) {  // rank order: deterministic
+                            const uint32_t peer = map_peer_smem(part_s, static_cast<uint32_t>(q));
+                            sg += ld_dsmem_f32(peer + static_cast<uint32_t>((m * 128 + row) * 4));
+                            su += ld_dsmem_f32(peer + static_cast<uint32_t>(((M + m) * 128 + row) * 4));
+                        }
+                        const float sx = (SCALED || !col_ok) ? 1.f : __ldg(p.sxf + m);
+                        dec_store_mxq(p, m, j, col_ok, lane,
+                                      dec_epi<SWIGLU, !SCALED>(p.epi, sg, su, sx, bgv, buv, wgv, wuv));
+                    }
+                }
+            }
             // one element per thread at a time: unrolling several (all their
             // remote loads first) measured slower, the larger code on this
             // short tail costing more than the round trips it saves
             constexpr int R = 1;
-            const int total_e = nrows * M;
+            const int total_e = (SWIGLU && p.q_codes) ? 0 : nrows * M;  // the MX-code output is done above
             for (int e0 = threadIdx.x; e0 < total_e; e0 += R * kDecThreads) {
                 float vg[R][8], vu[R][8];
                 float bg[R], bu[R], wg[R], wu[R], sx[R];
@@ -677,8 +727,8 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
                         }
                     }
                     if (j < p.Nout)
-                        p.out[static_cast<size_t>(m) * p.Nout + j] = __float2bfloat16_rn(
-                            dec_epi<SWIGLU, !SCALED>(p.epi, sg, su, sx[t], bg[t], bu[t], wg[t], wu[t]));
+                        store_out(p.out + static_cast<size_t>(m) * p.Nout + j, p.epi,
+                                  dec_epi<SWIGLU, !SCALED>(p.epi, sg, su, sx[t], bg[t], bu[t], wg[t], wu[t]));
                 }
             }
         }
@@ -864,7 +914,7 @@ size_t decode_ws_bytes(int tiles, int nsub, int M)
 // ring holds).  Returns false when the kernel cannot run the problem so.
 bool plan_decode(const GemmProblem& pb, int split, int grid, int cluster, int per_sm, int sms, GemmPlan* plan)
 {
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
+    const bool swiglu = epi_swiglu(pb.epi);
     const bool scaled = a_fmt_e8m0(pb.a_fmt);
     if (pb.M < 1 || pb.M > 64) return false;
     if (scaled && (pb.K % 128) != 0) return false;  // 4-byte scale copies
@@ -923,7 +973,7 @@ bool plan_decode(const GemmProblem& pb, int split, int grid, int cluster, int pe
 
 cudaError_t launch_decode(const GemmProblem& pb, const GemmPlan& plan, cudaStream_t st)
 {
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
+    const bool swiglu = epi_swiglu(pb.epi);
     const bool scaled = a_fmt_e8m0(pb.a_fmt);
     const bool e2m1 = pb.b_fmt == MX_B_E2M1_E8M0_1X32;
     const int mt = plan.block_m;
@@ -945,7 +995,13 @@ cudaError_t launch_decode(const GemmProblem& pb, const GemmPlan& plan, cudaStrea
     a.swf = scaled ? nullptr : static_cast<const float*>(pb.b_scales);
     a.sxf = scaled ? nullptr : static_cast<const float*>(pb.a_scales);
     a.bias = pb.bias;
-    a.out = static_cast<__nv_bfloat16*>(pb.out);
+    if (pb.epi == MX_EPI_SWIGLU_MXQ) {
+        // codes [M, N/2], then the E8M0 scales [M, N/64]
+        a.q_codes = static_cast<uint8_t*>(pb.out);
+        a.q_scales = a.q_codes + static_cast<size_t>(pb.M) * (pb.N / 2);
+    } else {
+        a.out = static_cast<__nv_bfloat16*>(pb.out);
+    }
     a.status = pb.status;
     if (plan.reduce) {
         uint8_t* ws = reinterpret_cast<uint8_t*>(pb.status);

@@ -21,7 +21,9 @@ struct DecodeArgs {
     const float* swf;    // per-channel fp32 weight scales [N]
     const float* sxf;    // per-token fp32 activation scales [M]
     const float* bias;   // fp32 [N] or null
-    __nv_bfloat16* out;  // [M, Nout]
+    __nv_bfloat16* out;  // [M, Nout] (null under MX_EPI_SWIGLU_MXQ)
+    uint8_t* q_codes;    // MX_EPI_SWIGLU_MXQ: e4m3 codes [M, Nout]
+    uint8_t* q_scales;   // MX_EPI_SWIGLU_MXQ: E8M0 scales [M, Nout / 32]
     unsigned* status;    // workspace status word
     unsigned* counters;  // [tiles] K blocks accumulated so far (zero between launches)
     float* red;          // [tiles][NSUB][M][128] fp32 accumulators (zero between launches)
@@ -93,6 +95,26 @@ __device__ __forceinline__ float dec_epi(int epi, float g, float u, float sx, fl
     if (epi == MX_EPI_NONE) return g;
     g += bg;
     return epi == MX_EPI_BIAS_GELU_TANH ? gelu_tanh(g) : g;
+}
+
+// MX_EPI_SWIGLU_MXQ: output value v of column j, token m, handed on as the
+// next GEMM's MX operand.  The 32 lanes of the calling warp hold 32
+// consecutive output columns of the same token -- one 1 x 32 block -- so the
+// block amax is a warp reduction; every lane of the warp must call this
+// (lanes outside the output pass col_ok = false and v = 0).  The value is
+// rounded to bf16 first, as the unfused chain stores it.
+__device__ __forceinline__ void dec_store_mxq(const DecodeArgs& p, int m, int j, bool col_ok, int lane, float v)
+{
+    const float vb = __bfloat162float(__float2bfloat16_rn(col_ok ? v : 0.f));
+    float amax = fabsf(vb);
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, s));
+    const int e = e8m0_exponent(amax, 8, 0x600000u);
+    const uint8_t code = static_cast<uint8_t>(to_e4m3x2(vb * pow2_neg(e), 0.f) & 0xFFu);
+    if (col_ok) {
+        p.q_codes[static_cast<size_t>(m) * p.Nout + j] = code;
+        if (lane == 0) p.q_scales[static_cast<size_t>(m) * (p.Nout / 32) + j / 32] = static_cast<uint8_t>(e);
+    }
 }
 
 // Fused activation quantisation: the token tile of each unit (M rows x 128 K)

@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2)
                                     if (j < p.Nout) {
                                         const float bg = p.bias ? __ldg(p.bias + j) : 0.f;
                                         const float bu = p.bias ? __ldg(p.bias + j + p.n_half) : 0.f;
-                                        orow[j] = __float2bfloat16_rn(dec_epi<true, false>(
+                                        store_out(orow + j, p.epi, dec_epi<true, false>(
                                             p.epi, __uint_as_float(gv[t]), __uint_as_float(uv[t]), 1.f, bg, bu, 1.f,
                                             1.f));
                                     }
@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2)
                                     const int j = tile * C::WROWS + c0 + t;
                                     if (j < p.Nout) {
                                         const float bg = p.bias ? __ldg(p.bias + j) : 0.f;
-                                        orow[j] = __float2bfloat16_rn(dec_epi<false, false>(
+                                        store_out(orow + j, p.epi, dec_epi<false, false>(
                                             p.epi, __uint_as_float(v[t]), 0.f, 1.f, bg, 0.f, 1.f, 1.f));
                                     }
                                 }
@@ -462,8 +462,8 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2)
                 if (j < p.Nout) {
                     const float bg = p.bias ? __ldg(p.bias + j) : 0.f;
                     const float bu = (SWIGLU && p.bias) ? __ldg(p.bias + j + p.n_half) : 0.f;
-                    p.out[static_cast<size_t>(m) * p.Nout + j] =
-                        __float2bfloat16_rn(dec_epi<SWIGLU, false>(p.epi, sg, su, 1.f, bg, bu, 1.f, 1.f));
+                    store_out(p.out + static_cast<size_t>(m) * p.Nout + j, p.epi,
+                              dec_epi<SWIGLU, false>(p.epi, sg, su, 1.f, bg, bu, 1.f, 1.f));
                 }
             }
         }
@@ -616,7 +616,7 @@ auto nw_dispatch(int mt, bool swiglu, bool one, const Op& op) -> decltype(op.inv
 // E8M0 formats; K % 128 == 0 (4-byte scale copies).
 bool plan_decode_nw(const GemmProblem& pb, int split, int grid, int cluster, int per_sm, GemmPlan* plan)
 {
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
+    const bool swiglu = epi_swiglu(pb.epi);
     if (!a_fmt_e8m0(pb.a_fmt) || pb.b_fmt == MX_B_E4M3_F32_ROW) return false;
     if (pb.M < 1 || pb.M > 64 || (pb.K % 128) != 0) return false;
     const int out_cols = swiglu ? kNwRows / 2 : kNwRows;
@@ -665,7 +665,7 @@ bool plan_decode_nw(const GemmProblem& pb, int split, int grid, int cluster, int
 
 cudaError_t launch_decode_nw(const GemmProblem& pb, const GemmPlan& plan, cudaStream_t st)
 {
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
+    const bool swiglu = epi_swiglu(pb.epi);
     const bool e2m1 = pb.b_fmt == MX_B_E2M1_E8M0_1X32;
     DecodeArgs a;
     memset(&a, 0, sizeof(a));

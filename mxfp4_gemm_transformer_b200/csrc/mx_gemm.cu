@@ -76,15 +76,21 @@ struct GemmArgs {
 //   128  one 128-row block per CTA tile;
 //   256  two 128-row blocks per CTA tile sharing each B tile (two M = 128 MMAs
 //        per K-step), halving the operand bytes each SM loads per FLOP.
-template <int BN, bool SCALED, bool SWIGLU, int AR = 128>
+template <int BN, int SC, bool SWIGLU, int AR = 128>
 struct Cfg {
+    static constexpr bool SCALED = SC != 0;  // E8M0 block scales (1: kind::mxf8f6f4, 2: kind::mxf4)
+    static constexpr bool F4 = SC == 2;      // both operands packed e2m1, K = 64 per MMA
     static constexpr int MB = AR == 256 ? 2 : 1;  // 128-row MMA blocks per tile
     static constexpr int BM = 128 * MB;
     static constexpr int BK = 128;  // K elements per stage (128 bytes per row in smem)
     static constexpr int A_BYTES = AR * BK;
     static constexpr int B_BYTES = BN * BK;
     static constexpr int SFB_CHUNKS = (BN + 127) / 128;
-    static constexpr int SF_BYTES = SCALED ? 512 * (MB + SFB_CHUNKS) : 0;
+    // K elements per stage: 128 one-byte codes per row, or 256 packed e2m1
+    // (kind::mxf4), whose stage then carries two scale chunks of 4 K blocks
+    static constexpr int KPS = F4 ? 256 : 128;
+    static constexpr int SF_CHUNK = 512 * (MB + SFB_CHUNKS);
+    static constexpr int SF_BYTES = SCALED ? SF_CHUNK * (F4 ? 2 : 1) : 0;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024) * 1024;
     static constexpr int SMEM_LIMIT = 232448;
     // output staging: one 32 x 32 bf16 chunk per epilogue warp, transposed through
@@ -201,7 +207,7 @@ __device__ __forceinline__ float epi_apply(const EpiCtx& c, float g, float u, co
 
 // value of output column n from gate/plain accumulator g and up accumulator u
 template <bool SWIGLU>
-__device__ __forceinline__ float epi_value(const EpiCtx& c, float g, float u, int n)
+__device__ __forceinline__ float epi_value(const EpiCtx& c, float g, float u, int n, float res = 0.f)
 {
     if (c.f32row) {
         g *= c.sx * __ldcg(c.swb + n);
@@ -215,7 +221,8 @@ __device__ __forceinline__ float epi_value(const EpiCtx& c, float g, float u, in
         return sigmoid_mul(g, g) * u;
     }
     if (c.epi == MX_EPI_NONE) return g;
-    g += __ldcg(c.bias + n);
+    if (c.bias) g += __ldcg(c.bias + n);
+    if (c.epi == MX_EPI_RESIDUAL) return g + res;
     return c.epi == MX_EPI_BIAS_GELU_TANH ? gelu_tanh(g) : g;
 }
 
@@ -223,10 +230,12 @@ constexpr int kThreads = 128 + kEpiThreads;
 
 // ---------------------------------------------------------------------------
 
-template <int BN, bool SCALED, bool SWIGLU, int AR>
+template <int BN, int SC, bool SWIGLU, int AR>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs p)
 {
-    using C = Cfg<BN, SCALED, SWIGLU, AR>;
+    using C = Cfg<BN, SC, SWIGLU, AR>;
+    constexpr bool SCALED = C::SCALED;
+    constexpr bool F4 = C::F4;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
@@ -367,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     stamp_stage(p, 1, dbg_i);
                     const uint32_t sA = smem_u32(ring + stage * C::STAGE_BYTES);
                     const uint32_t sB = sA + C::A_BYTES;
-                    if (SCALED) {
+                    if (SCALED && !F4) {
                         const uint32_t sf = sB + C::B_BYTES;
 #pragma unroll
                         for (int rb = 0; rb < C::MB; ++rb) tc_cp_32x128b_x4(tmem_sfa + 4 * rb, sdesc_sf(sf + 512 * rb));
@@ -375,18 +384,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                         for (int j = 0; j < C::SFB_CHUNKS; ++j)
                             tc_cp_32x128b_x4(tmem_sfb + 4 * j, sdesc_sf(sf + 512 * (C::MB + j)));
                     }
-                    const int krem = p.K - kb * C::BK;
-                    const int ksteps = krem >= C::BK ? 4 : krem / 32;
+                    const int krem = p.K - kb * C::KPS;
+                    const int ksteps = F4 ? (krem >= 256 ? 4 : krem / 64) : (krem >= C::BK ? 4 : krem / 32);
                     for (int kk = 0; kk < ksteps; ++kk) {
+                        if (F4 && (kk & 1) == 0) {
+                            // one scale chunk (4 K blocks of 32) per two K = 64 MMAs; the
+                            // copy is ordered after the previous MMAs that read the columns
+                            const uint32_t sf = sB + C::B_BYTES + (kk >> 1) * C::SF_CHUNK;
+#pragma unroll
+                            for (int rb = 0; rb < C::MB; ++rb)
+                                tc_cp_32x128b_x4(tmem_sfa + 4 * rb, sdesc_sf(sf + 512 * rb));
+#pragma unroll
+                            for (int j = 0; j < C::SFB_CHUNKS; ++j)
+                                tc_cp_32x128b_x4(tmem_sfb + 4 * j, sdesc_sf(sf + 512 * (C::MB + j)));
+                        }
                         const uint64_t bd = sdesc_sw128(sB + kk * 32);
 #pragma unroll
                         for (int rb = 0; rb < C::MB; ++rb) {
                             const uint64_t ad = sdesc_sw128(sA + rb * 16384 + kk * 32);
                             const uint32_t drb = d + rb * C::RB_STRIDE;
                             if (SCALED) {
-                                const uint32_t id = p.idesc | (static_cast<uint32_t>(kk) << 4) |
-                                                    (static_cast<uint32_t>(kk) << 29);
-                                mma_mx(drb, ad, bd, id, tmem_sfa + 4 * rb, tmem_sfb, accumulate);
+                                // scale id: the byte (or, for kind::mxf4, the byte pair)
+                                // of the chunk's 32-bit column this MMA's K blocks use
+                                const uint32_t sid = F4 ? static_cast<uint32_t>((kk & 1) * 2) : static_cast<uint32_t>(kk);
+                                const uint32_t id = p.idesc | (sid << 4) | (sid << 29);
+                                if (F4) mma_mxf4(drb, ad, bd, id, tmem_sfa + 4 * rb, tmem_sfb, accumulate);
+                                else mma_mx(drb, ad, bd, id, tmem_sfa + 4 * rb, tmem_sfb, accumulate);
                             } else {
                                 mma_f8(drb, ad, bd, p.idesc, accumulate);
                             }
@@ -464,8 +487,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 const int tn = tile / p.tiles_m;
                 const int kb0 = split * p.num_kb / p.splits, kb1 = (split + 1) * p.num_kb / p.splits;
                 pre = min(C::STAGES, kb1 - kb0);
-                for (int i = 0; i < pre; ++i)
-                    issue_b(ring + i * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES, tn, (kb0 + i) * 4);
+                for (int i = 0; i < pre; ++i) {
+                    uint8_t* sf = ring + i * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+                    const int kbase = (kb0 + i) * (C::KPS / 32);
+#pragma unroll
+                    for (int c = 0; c < (F4 ? 2 : 1); ++c)
+                        if (kbase + 4 * c < KB) issue_b(sf + c * C::SF_CHUNK, tn, kbase + 4 * c);
+                }
             }
             pdl_wait();
             for (int u = u_first; u < p.units; u += u_step) {
@@ -474,14 +502,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 const int kb0 = split * p.num_kb / p.splits, kb1 = (split + 1) * p.num_kb / p.splits;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     uint8_t* sf = ring + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
-                    const int k4 = kb * 4;  // first 32-wide K block of this stage
+                    const int k4 = kb * (C::KPS / 32);  // first 32-wide K block of this stage
                     if (pre > 0) {
                         --pre;
-                        issue_a(sf, tm, k4);
+#pragma unroll
+                        for (int c = 0; c < (F4 ? 2 : 1); ++c)
+                            if (k4 + 4 * c < KB) issue_a(sf + c * C::SF_CHUNK, tm, k4 + 4 * c);
                         cp_async_arrive_noinc(&full[stage]);
                     } else {
                         if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.status)) goto sf_done;
-                        if (vec4) {
+                        if (F4) {
+                            // two chunks of 4 K blocks; a chunk wholly past K is not
+                            // read (its MMAs are not issued)
+#pragma unroll
+                            for (int c = 0; c < 2; ++c)
+                                if (k4 + 4 * c < KB) {
+                                    issue_a(sf + c * C::SF_CHUNK, tm, k4 + 4 * c);
+                                    issue_b(sf + c * C::SF_CHUNK, tn, k4 + 4 * c);
+                                }
+                            cp_async_arrive_noinc(&full[stage]);
+                        } else if (vec4) {
                             issue_a(sf, tm, k4);
                             issue_b(sf, tn, k4);
                             cp_async_arrive_noinc(&full[stage]);
@@ -667,14 +707,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                         __nv_bfloat16* o = p.out + static_cast<size_t>(m) * p.Nout + n0;
                         if (n0 + 4 <= p.Nout && (p.Nout & 3) == 0) {
                             uint2 v2;
-                            v2.x = pack_bf16x2(epi_value<SWIGLU>(ec, gv[0], uv[0], n0),
-                                               epi_value<SWIGLU>(ec, gv[1], uv[1], n0 + 1));
-                            v2.y = pack_bf16x2(epi_value<SWIGLU>(ec, gv[2], uv[2], n0 + 2),
-                                               epi_value<SWIGLU>(ec, gv[3], uv[3], n0 + 3));
+                            float rv[4] = {0.f, 0.f, 0.f, 0.f};
+                            if (p.epi == MX_EPI_RESIDUAL) {
+                                const uint2 q2 = *reinterpret_cast<const uint2*>(o);
+                                rv[0] = __uint_as_float(q2.x << 16);
+                                rv[1] = __uint_as_float(q2.x & 0xFFFF0000u);
+                                rv[2] = __uint_as_float(q2.y << 16);
+                                rv[3] = __uint_as_float(q2.y & 0xFFFF0000u);
+                            }
+                            v2.x = pack_bf16x2(epi_value<SWIGLU>(ec, gv[0], uv[0], n0, rv[0]),
+                                               epi_value<SWIGLU>(ec, gv[1], uv[1], n0 + 1, rv[1]));
+                            v2.y = pack_bf16x2(epi_value<SWIGLU>(ec, gv[2], uv[2], n0 + 2, rv[2]),
+                                               epi_value<SWIGLU>(ec, gv[3], uv[3], n0 + 3, rv[3]));
                             *reinterpret_cast<uint2*>(o) = v2;
                         } else {
                             for (int j = 0; j < 4; ++j)
-                                if (n0 + j < p.Nout) o[j] = __float2bfloat16_rn(epi_value<SWIGLU>(ec, gv[j], uv[j], n0 + j));
+                                if (n0 + j < p.Nout) store_out(o + j, p.epi, epi_value<SWIGLU>(ec, gv[j], uv[j], n0 + j));
                         }
                     }
                 }
@@ -717,6 +765,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     } else if (p.epi == MX_EPI_BIAS) {
                         if (f32row) epi_chunk<MX_EPI_BIAS, false, true>(g, h, sx, colp, c, pk);
                         else epi_chunk<MX_EPI_BIAS, false, false>(g, h, sx, colp, c, pk);
+                    } else if (p.epi == MX_EPI_RESIDUAL) {
+                        float res[32];
+                        load_row32_bf16(p.out, p.Nout, p.M, m, n_base + c, min(min(32, C::OUT_COLS - c), p.Nout - (n_base + c)),
+                                        res);
+                        if (f32row) epi_chunk_residual<true>(g, sx, colp, c, res, pk);
+                        else epi_chunk_residual<false>(g, sx, colp, c, res, pk);
                     } else {
                         if (f32row) epi_chunk<MX_EPI_NONE, false, true>(g, h, sx, colp, c, pk);
                         else epi_chunk<MX_EPI_NONE, false, false>(g, h, sx, colp, c, pk);
@@ -804,12 +858,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 __nv_bfloat16* dst = p.out + static_cast<size_t>(m) * p.Nout + n0;
                 if (n0 + 4 <= p.Nout && (p.Nout & 3) == 0) {
                     uint2 o;
-                    o.x = pack_bf16x2(epi_value<SWIGLU>(ec, gv[0], uv[0], n0), epi_value<SWIGLU>(ec, gv[1], uv[1], n0 + 1));
-                    o.y = pack_bf16x2(epi_value<SWIGLU>(ec, gv[2], uv[2], n0 + 2), epi_value<SWIGLU>(ec, gv[3], uv[3], n0 + 3));
+                    float rv[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (p.epi == MX_EPI_RESIDUAL) {
+                        const uint2 q2 = *reinterpret_cast<const uint2*>(dst);
+                        rv[0] = __uint_as_float(q2.x << 16);
+                        rv[1] = __uint_as_float(q2.x & 0xFFFF0000u);
+                        rv[2] = __uint_as_float(q2.y << 16);
+                        rv[3] = __uint_as_float(q2.y & 0xFFFF0000u);
+                    }
+                    o.x = pack_bf16x2(epi_value<SWIGLU>(ec, gv[0], uv[0], n0, rv[0]),
+                                      epi_value<SWIGLU>(ec, gv[1], uv[1], n0 + 1, rv[1]));
+                    o.y = pack_bf16x2(epi_value<SWIGLU>(ec, gv[2], uv[2], n0 + 2, rv[2]),
+                                      epi_value<SWIGLU>(ec, gv[3], uv[3], n0 + 3, rv[3]));
                     *reinterpret_cast<uint2*>(dst) = o;
                 } else {
                     for (int j = 0; j < 4; ++j)
-                        if (n0 + j < p.Nout) dst[j] = __float2bfloat16_rn(epi_value<SWIGLU>(ec, gv[j], uv[j], n0 + j));
+                        if (n0 + j < p.Nout) store_out(dst + j, p.epi, epi_value<SWIGLU>(ec, gv[j], uv[j], n0 + j));
                 }
             }
         }
@@ -903,11 +967,11 @@ int g_timeline_ctas = 0;
 
 // Kernel attributes are per device: set them the first time a device uses
 // this kernel (before any stream capture, since the first call is eager).
-template <int BN, bool SCALED, bool SWIGLU, int AR>
+template <int BN, int SC, bool SWIGLU, int AR>
 cudaError_t prepare_kernel()
 {
-    using C = Cfg<BN, SCALED, SWIGLU, AR>;
-    auto kern = gemm_kernel<BN, SCALED, SWIGLU, AR>;
+    using C = Cfg<BN, SC, SWIGLU, AR>;
+    auto kern = gemm_kernel<BN, SC, SWIGLU, AR>;
     static std::mutex mu;
     static bool done[64] = {};
     int dev = 0;
@@ -923,14 +987,17 @@ cudaError_t prepare_kernel()
     return cudaSuccess;
 }
 
-// The compiled variants: (tile width, activation rows) x scaled x SwiGLU.
+// The compiled variants: (tile width, activation rows) x scaling (sc: 0 fp32
+// row / column scales, 1 E8M0 kind::mxf8f6f4, 2 E8M0 kind::mxf4 W4A4) x SwiGLU.
 template <class Op>
-auto dispatch(int bn, int ar, bool scaled, bool swiglu, Op op) -> decltype(op.template run<128, true, false, 128>())
+auto dispatch(int bn, int ar, int sc, bool swiglu, Op op) -> decltype(op.template run<128, 1, false, 128>())
 {
 #define MXG_DISPATCH(B, A)                                                                                    \
-    if (bn == B && ar == A)                                                                                   \
-        return scaled ? (swiglu ? op.template run<B, true, true, A>() : op.template run<B, true, false, A>())   \
-                      : (swiglu ? op.template run<B, false, true, A>() : op.template run<B, false, false, A>());
+    if (bn == B && ar == A && sc != 2)                                                                        \
+        return sc ? (swiglu ? op.template run<B, 1, true, A>() : op.template run<B, 1, false, A>())             \
+                  : (swiglu ? op.template run<B, 0, true, A>() : op.template run<B, 0, false, A>());
+#define MXG_DISPATCH_F4(B, A)                                                                                 \
+    if (bn == B && ar == A && sc == 2) return swiglu ? op.template run<B, 2, true, A>() : op.template run<B, 2, false, A>();
     MXG_DISPATCH(64, 128)
     MXG_DISPATCH(128, 128)
     MXG_DISPATCH(240, 128)
@@ -938,21 +1005,25 @@ auto dispatch(int bn, int ar, bool scaled, bool swiglu, Op op) -> decltype(op.te
     MXG_DISPATCH(128, 64)
     MXG_DISPATCH(256, 64)
     MXG_DISPATCH(240, 256)
+    MXG_DISPATCH_F4(240, 128)
+    MXG_DISPATCH_F4(256, 128)
+    MXG_DISPATCH_F4(240, 256)
 #undef MXG_DISPATCH
+#undef MXG_DISPATCH_F4
     return op.invalid();
 }
 
 struct AccBufsOp {
-    template <int BN, bool SCALED, bool SWIGLU, int AR>
-    int run() const { return Cfg<BN, SCALED, SWIGLU, AR>::ACC_BUFS; }
+    template <int BN, int SC, bool SWIGLU, int AR>
+    int run() const { return Cfg<BN, SC, SWIGLU, AR>::ACC_BUFS; }
     int invalid() const { return 0; }
 };
 
 struct RingOp {
-    template <int BN, bool SCALED, bool SWIGLU, int AR>
+    template <int BN, int SC, bool SWIGLU, int AR>
     long long run() const
     {
-        return static_cast<long long>(Cfg<BN, SCALED, SWIGLU, AR>::STAGES) * Cfg<BN, SCALED, SWIGLU, AR>::STAGE_BYTES;
+        return static_cast<long long>(Cfg<BN, SC, SWIGLU, AR>::STAGES) * Cfg<BN, SC, SWIGLU, AR>::STAGE_BYTES;
     }
     long long invalid() const { return 0; }
 };
@@ -961,10 +1032,10 @@ struct RingOp {
 // once (cached per device, variant and cluster size).
 struct ClustersOp {
     int cluster;
-    template <int BN, bool SCALED, bool SWIGLU, int AR>
+    template <int BN, int SC, bool SWIGLU, int AR>
     int run() const
     {
-        using C = Cfg<BN, SCALED, SWIGLU, AR>;
+        using C = Cfg<BN, SC, SWIGLU, AR>;
         static std::mutex mu;
         static int cache[64][17] = {};
         int dev = 0;
@@ -973,7 +1044,7 @@ struct ClustersOp {
             std::lock_guard<std::mutex> lk(mu);
             if (cache[dev][cluster]) return cache[dev][cluster];
         }
-        if (prepare_kernel<BN, SCALED, SWIGLU, AR>() != cudaSuccess) return 0;
+        if (prepare_kernel<BN, SC, SWIGLU, AR>() != cudaSuccess) return 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(cluster * 64, 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
@@ -986,7 +1057,7 @@ struct ClustersOp {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<BN, SCALED, SWIGLU, AR>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<BN, SC, SWIGLU, AR>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -997,15 +1068,15 @@ struct ClustersOp {
     int invalid() const { return 0; }
 };
 
-int max_active_clusters_for(int bn, int ar, bool scaled, bool swiglu, int cluster)
+int max_active_clusters_for(int bn, int ar, int sc, bool swiglu, int cluster)
 {
-    return dispatch(bn, ar, scaled, swiglu, ClustersOp{cluster});
+    return dispatch(bn, ar, sc, swiglu, ClustersOp{cluster});
 }
 
 // Whether the parked split-K partial (rows x (BN + 4) fp32) fits in the ring.
-bool split_fits(int bn, int ar, bool scaled, bool swiglu, int rows)
+bool split_fits(int bn, int ar, int sc, bool swiglu, int rows)
 {
-    const long long ring = dispatch(bn, ar, scaled, swiglu, RingOp{});
+    const long long ring = dispatch(bn, ar, sc, swiglu, RingOp{});
     return ring > 0 && static_cast<long long>(rows) * (bn + 4) * 4 <= ring;
 }
 
@@ -1013,12 +1084,12 @@ struct LaunchOp {
     const GemmArgs* args;
     const GemmPlan* plan;
     cudaStream_t st;
-    template <int BN, bool SCALED, bool SWIGLU, int AR>
+    template <int BN, int SC, bool SWIGLU, int AR>
     cudaError_t run() const
     {
-        using C = Cfg<BN, SCALED, SWIGLU, AR>;
-        auto kern = gemm_kernel<BN, SCALED, SWIGLU, AR>;
-        cudaError_t e = prepare_kernel<BN, SCALED, SWIGLU, AR>();
+        using C = Cfg<BN, SC, SWIGLU, AR>;
+        auto kern = gemm_kernel<BN, SC, SWIGLU, AR>;
+        cudaError_t e = prepare_kernel<BN, SC, SWIGLU, AR>();
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(plan->grid_x, plan->grid_y, 1);
@@ -1048,8 +1119,8 @@ struct LaunchOp {
 
 
 struct StagesOp {
-    template <int BN, bool SCALED, bool SWIGLU, int AR>
-    int run() const { return Cfg<BN, SCALED, SWIGLU, AR>::STAGES; }
+    template <int BN, int SC, bool SWIGLU, int AR>
+    int run() const { return Cfg<BN, SC, SWIGLU, AR>::STAGES; }
     int invalid() const { return 0; }
 };
 
@@ -1120,6 +1191,29 @@ size_t gsplit_ws_bytes(int tiles, int splits, int part_rows, int bn)
 // split counts, take the one with the lowest estimated time.
 cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_bytes, GemmPlan* plan)
 {
+    if (pb.epi == MX_EPI_SWIGLU_MXQ) {
+        // The SwiGLU GEMM whose output is handed on as MX codes: quantised in
+        // the decode kernel's epilogue (a warp's lanes hold one 1 x 32 block
+        // of a token), else stored as bf16 into the workspace behind what the
+        // plan needs and quantised from there by the activation quantiser.
+        GemmProblem q = pb;
+        q.epi = MX_EPI_SWIGLU;
+        cudaError_t e = plan_gemm(q, dev, ws_bytes, plan);
+        if (e != cudaSuccess) return e;
+        if (plan->kernel == 1) {
+            plan->out_quant = 1;
+            return cudaSuccess;
+        }
+        const size_t tbytes = static_cast<size_t>(pb.M) * (pb.N / 2) * 2;
+        const size_t avail = ws_bytes > tbytes + kWorkspaceHeader ? ws_bytes - tbytes : kWorkspaceHeader;
+        *plan = GemmPlan();
+        e = plan_gemm(q, dev, avail, plan);
+        if (e != cudaSuccess) return e;
+        plan->out_quant = 2;
+        plan->out_off = (plan->ws_bytes + 255) / 256 * 256;
+        plan->ws_bytes = plan->out_off + tbytes;
+        return cudaSuccess;
+    }
     if (pb.a_fmt == MX_A_BF16_E8M0_1X32) {
         // bf16 activations: the plan for the equivalent codes.  The codes are
         // made once, into the workspace behind what the plan needs, by the
@@ -1155,8 +1249,9 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
         }
         return cudaSuccess;
     }
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
-    const bool scaled = pb.a_fmt == MX_A_E4M3_E8M0_1X32;
+    const bool swiglu = epi_swiglu(pb.epi);
+    const int sc = pb.a_fmt == MX_A_E4M3_E8M0_1X32 ? 1 : (pb.a_fmt == MX_A_E2M1_E8M0_1X32 ? 2 : 0);
+    const bool scaled = sc != 0;
     const int nout = swiglu ? pb.N / 2 : pb.N;
     const int num_kb = (pb.K + 127) / 128;
     const int tiles_m = (pb.M + 127) / 128;
@@ -1180,7 +1275,7 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
     // All of these are deterministic and need no workspace; the stream-K
     // split (workspace atomics) is used only when asked for.
     const bool tuned = g_tune_bn != 0 || g_tune_splits != 0 || g_tune_bm != 0 || g_tune_ctas != 0;
-    if (pb.M <= 64 && g_dec_mode >= 0 && (g_dec_mode >= 1 || !tuned)) {
+    if (pb.M <= 64 && g_dec_mode >= 0 && (g_dec_mode >= 1 || !tuned) && sc != 2) {
         const bool det = (launch_flags() & MX_LAUNCH_DETERMINISTIC) != 0;
         // On request (mode 2), for E8M0 formats: the kernel with the weights
         // on the MMA's N side (240 weight rows per instruction, 1.9x the
@@ -1245,7 +1340,7 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
     }
 
     // 256 x 240 tiles over CTA pairs (cta_group::2 MMAs), on request
-    if (g_tune_bm == kTuneBmPair && g_tune_splits <= 1 && (g_tune_bn == 0 || g_tune_bn == 240) &&
+    if (g_tune_bm == kTuneBmPair && g_tune_splits <= 1 && (g_tune_bn == 0 || g_tune_bn == 240) && sc != 2 &&
         plan_pair(pb, sms, g_tune_ctas, plan))
         return cudaSuccess;
 
@@ -1300,8 +1395,8 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
                         tail = 3000.0 + static_cast<double>(s) * part_rows * b * 4 / reduce_bytes_per_cycle;
                     } else if (s > 1) {
                         if (s > 16) continue;
-                        if (max_active_clusters_for(b, ar, scaled, swiglu, s) < t) continue;
-                        if (!split_fits(b, ar, scaled, swiglu, pb.M)) continue;
+                        if (max_active_clusters_for(b, ar, sc, swiglu, s) < t) continue;
+                        if (!split_fits(b, ar, sc, swiglu, pb.M)) continue;
                         tail = 2500.0 + static_cast<double>(part_rows) * b * 4 / reduce_bytes_per_cycle;
                     } else if (g == 1) {
                         continue;
@@ -1321,12 +1416,19 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
         gsplit = best_g;
     }
     if (splits < 1) splits = 1;
+    if (sc == 2) {
+        // W4A4 (kind::mxf4): compiled for 240- and 256-wide tiles of 128 or
+        // 256 rows, without K splits
+        bn = g_tune_bn == 256 ? 256 : 240;
+        splits = 1;
+    }
     if (splits == 1) gsplit = 0;
 
     // Tile height: two 128-row blocks per tile (halving operand bytes per FLOP)
     // when K is not split, the tile is 240 wide and there are at least as many
     // 256-row tiles as SMs; 64 loaded rows for decode-sized M.
     int a_rows = ar_for(bn);
+    if (sc == 2) a_rows = 128;
     const int oc = swiglu ? bn / 2 : bn;
     const int tiles_n = (nout + oc - 1) / oc;
     const bool tall_ok = splits == 1 && bn == 240;
@@ -1345,8 +1447,8 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
     plan->part_rows = gsplit ? part_rows : 0;
     plan->ws_bytes = gsplit ? gsplit_ws_bytes(tiles, splits, part_rows, bn) : kWorkspaceHeader;
     plan->units = tiles * splits;
-    plan->acc_bufs = dispatch(bn, a_rows, scaled, swiglu, AccBufsOp{});
-    plan->stages = dispatch(bn, a_rows, scaled, swiglu, StagesOp{});
+    plan->acc_bufs = dispatch(bn, a_rows, sc, swiglu, AccBufsOp{});
+    plan->stages = dispatch(bn, a_rows, sc, swiglu, StagesOp{});
     if (splits > 1 && !gsplit) {
         plan->grid_x = splits;
         plan->grid_y = tiles;
@@ -1376,21 +1478,45 @@ cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_
         p2.act_quant = 0;
         return launch_gemm(q, p2, st);
     }
+    if (plan.out_quant == 2) {
+        // SwiGLU into the workspace as bf16, then its 1 x 32 quantisation into
+        // out (codes, then scales)
+        uint8_t* ws = reinterpret_cast<uint8_t*>(pb.status);
+        __nv_bfloat16* tmp = reinterpret_cast<__nv_bfloat16*>(ws + plan.out_off);
+        GemmProblem q = pb;
+        q.epi = MX_EPI_SWIGLU;
+        q.out = tmp;
+        GemmPlan p2 = plan;
+        p2.out_quant = 0;
+        cudaError_t e = launch_gemm(q, p2, st);
+        if (e != cudaSuccess) return e;
+        uint8_t* codes = static_cast<uint8_t*>(pb.out);
+        return launch_quant_e8m0_1x32(tmp, pb.M, pb.N / 2, codes, codes + static_cast<size_t>(pb.M) * (pb.N / 2), st);
+    }
     if (plan.kernel == 1) return launch_decode(pb, plan, st);
     if (plan.kernel == 2) return launch_decode_nw(pb, plan, st);
     if (plan.kernel == 3) return launch_pair(pb, plan, st);
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
-    const bool scaled = pb.a_fmt == MX_A_E4M3_E8M0_1X32;
+    const bool swiglu = epi_swiglu(pb.epi);
+    const int sc = pb.a_fmt == MX_A_E4M3_E8M0_1X32 ? 1 : (pb.a_fmt == MX_A_E2M1_E8M0_1X32 ? 2 : 0);
+    const bool scaled = sc != 0;
     const int bn = plan.block_n;
     const int out_cols = swiglu ? bn / 2 : bn;
 
     GemmArgs a;
     memset(&a, 0, sizeof(a));
-    if (!make_map(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.a_codes, pb.K, pb.M, pb.K, 128,
-                  static_cast<uint32_t>(plan.a_rows)))
-        return cudaErrorInvalidValue;
+    const bool f4 = pb.a_fmt == MX_A_E2M1_E8M0_1X32;  // W4A4, kind::mxf4
     const uint32_t b_rows = swiglu ? bn / 2 : bn;
-    if (pb.b_fmt == MX_B_E2M1_E8M0_1X32) {
+    if (f4) {
+        // both operands packed two per byte, loaded as plain bytes: a 128-byte
+        // row of a stage holds 256 K elements
+        if (!make_map(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.a_codes, pb.K / 2, pb.M, pb.K / 2, 128,
+                      static_cast<uint32_t>(plan.a_rows)) ||
+            !make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.b_codes, pb.K / 2, pb.N, pb.K / 2, 128, b_rows))
+            return cudaErrorInvalidValue;
+    } else if (!make_map(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.a_codes, pb.K, pb.M, pb.K, 128,
+                         static_cast<uint32_t>(plan.a_rows))) {
+        return cudaErrorInvalidValue;
+    } else if (pb.b_fmt == MX_B_E2M1_E8M0_1X32) {
         if (!make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, pb.b_codes, pb.K, pb.N, pb.K / 2, 128, b_rows))
             return cudaErrorInvalidValue;
     } else {
@@ -1420,7 +1546,7 @@ cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_
     a.K = pb.K;
     a.Nout = swiglu ? pb.N / 2 : pb.N;
     a.KB = pb.K / 32;
-    a.num_kb = (pb.K + 127) / 128;
+    a.num_kb = f4 ? (pb.K + 255) / 256 : (pb.K + 127) / 128;
     a.tiles_m = (pb.M + plan.block_m - 1) / plan.block_m;
     a.tiles_n = (a.Nout + out_cols - 1) / out_cols;
     a.splits = plan.splits;
@@ -1429,7 +1555,10 @@ cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_
     a.epi = pb.epi;
     a.n_half = pb.N / 2;
     const uint32_t b_code = (pb.b_fmt == MX_B_E2M1_E8M0_1X32) ? 5u : 0u;  // e2m1 : e4m3
-    if (scaled)
+    if (f4)  // kind::mxf4: E2M1 is format 1 for both operands; K = 64 per MMA
+        a.idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | (1u << 23) |
+                  (static_cast<uint32_t>(128 >> 4) << 24);
+    else if (scaled)
         a.idesc = (0u << 7) | (b_code << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | (1u << 23) |
                   (static_cast<uint32_t>(128 >> 4) << 24);
     else
@@ -1438,10 +1567,10 @@ cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_
     // transaction bytes count the global-side size: a 128-element e2m1 row is
     // 64 bytes even though it lands as 128 bytes (16 codes + 8 pad bytes per
     // 16-byte chunk) in shared memory
-    const uint32_t b_row_bytes = (pb.b_fmt == MX_B_E2M1_E8M0_1X32) ? 64u : 128u;
+    const uint32_t b_row_bytes = (pb.b_fmt == MX_B_E2M1_E8M0_1X32 && !f4) ? 64u : 128u;
     a.tx_bytes = static_cast<uint32_t>(plan.a_rows * 128) + static_cast<uint32_t>(bn) * b_row_bytes;
 
-    return dispatch(bn, plan.a_rows, scaled, swiglu, LaunchOp{&a, &plan, st});
+    return dispatch(bn, plan.a_rows, sc, swiglu, LaunchOp{&a, &plan, st});
 }
 
 }  // namespace mxg

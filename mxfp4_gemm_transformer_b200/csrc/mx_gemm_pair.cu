@@ -440,6 +440,12 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
                     } else if (p.epi == MX_EPI_BIAS) {
                         if (f32row) epi_chunk<MX_EPI_BIAS, false, true>(g, h, sx, colp, c, pk);
                         else epi_chunk<MX_EPI_BIAS, false, false>(g, h, sx, colp, c, pk);
+                    } else if (p.epi == MX_EPI_RESIDUAL) {
+                        float res[32];
+                        load_row32_bf16(p.out, p.Nout, p.M, m, n_base + c,
+                                        min(min(32, C::OUT_COLS - c), p.Nout - (n_base + c)), res);
+                        if (f32row) epi_chunk_residual<true>(g, sx, colp, c, res, pk);
+                        else epi_chunk_residual<false>(g, sx, colp, c, res, pk);
                     } else {
                         if (f32row) epi_chunk<MX_EPI_NONE, false, true>(g, h, sx, colp, c, pk);
                         else epi_chunk<MX_EPI_NONE, false, false>(g, h, sx, colp, c, pk);
@@ -575,7 +581,7 @@ int max_active_pairs(bool scaled, bool swiglu)
 
 bool plan_pair(const GemmProblem& pb, int sms, int max_ctas, GemmPlan* plan)
 {
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
+    const bool swiglu = epi_swiglu(pb.epi);
     const bool scaled = pb.a_fmt == MX_A_E4M3_E8M0_1X32;
     const int nout = swiglu ? pb.N / 2 : pb.N;
     const int out_cols = swiglu ? 120 : 240;
@@ -604,7 +610,7 @@ bool plan_pair(const GemmProblem& pb, int sms, int max_ctas, GemmPlan* plan)
 
 cudaError_t launch_pair(const GemmProblem& pb, const GemmPlan& plan, cudaStream_t st)
 {
-    const bool swiglu = pb.epi == MX_EPI_SWIGLU;
+    const bool swiglu = epi_swiglu(pb.epi);
     const bool scaled = pb.a_fmt == MX_A_E4M3_E8M0_1X32;
     PairArgs a;
     memset(&a, 0, sizeof(a));

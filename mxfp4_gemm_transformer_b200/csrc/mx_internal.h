@@ -9,6 +9,9 @@
 
 namespace mxg {
 
+// Epilogues whose weight is a fused [gate; up] with N rows and N/2 outputs.
+inline bool epi_swiglu(int epi) { return epi == MX_EPI_SWIGLU || epi == MX_EPI_SWIGLU_MXQ; }
+
 // Status word bits written by kernels into the workspace.
 constexpr unsigned kStatusTimeout = 1u;
 
@@ -35,6 +38,8 @@ struct DeviceInfo {
 cudaError_t current_device(DeviceInfo* out);
 
 // ---- quantisation launchers (mx_quant.cu) ---------------------------------
+cudaError_t launch_add_rms_quant(const void* x, void* res, const void* w, float eps, int M, int K, void* y_out,
+                                 void* codes, void* scales, cudaStream_t st);
 cudaError_t launch_quant_e8m0_1x32(const void* x, long long rows, int K, uint8_t* codes, uint8_t* scales,
                                    cudaStream_t st);
 cudaError_t launch_quant_f32_row(const void* x, int rows, int K, uint8_t* codes, float* scales, cudaStream_t st);
@@ -106,6 +111,11 @@ struct GemmPlan {
     // quantisation kernel before the GEMM (act_quant = 2)
     int act_quant = 0;
     size_t quant_off = 0;
+    // MX_EPI_SWIGLU_MXQ: the SwiGLU output quantised inside the decode
+    // kernel's epilogue (out_quant = 1), or stored as bf16 into the workspace
+    // at byte out_off and quantised from there (out_quant = 2)
+    int out_quant = 0;
+    size_t out_off = 0;
 };
 
 // How the decode kernel shares a tile's K range between CTAs.

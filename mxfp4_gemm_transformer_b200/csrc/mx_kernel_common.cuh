@@ -107,6 +107,62 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&g)[32], const uint32_
 }
 
 
+// The in-place residual epilogue of one 32-column chunk: acc (x row/column
+// fp32 scales) + bias (0 without one) + the residual already in out, rounded
+// once to bf16 pairs.
+template <bool F32ROW>
+__device__ __forceinline__ void epi_chunk_residual(const uint32_t (&g)[32], float sx, const float* __restrict__ colp,
+                                                   int c, const float (&res)[32], uint32_t (&packed)[16])
+{
+#pragma unroll
+    for (int j2 = 0; j2 < 16; ++j2) {
+        float v[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const int j = 2 * j2 + t;
+            float a = __uint_as_float(g[j]);
+            if (F32ROW) a *= sx * colp[512 + c + j];
+            v[t] = (a + colp[c + j]) + res[j];
+        }
+        packed[j2] = pack_bf16x2(v[0], v[1]);
+    }
+}
+
+// out[m, col0 .. col0 + 31] as fp32, the residual the in-place epilogue adds
+// (zeros past the `lim` valid columns, or for rows >= M).
+__device__ __forceinline__ void load_row32_bf16(const __nv_bfloat16* out, int Nout, int M, int m, int col0, int lim,
+                                                float (&r)[32])
+{
+#pragma unroll
+    for (int j = 0; j < 32; ++j) r[j] = 0.f;
+    if (m >= M || lim <= 0) return;
+    const __nv_bfloat16* src = out + static_cast<size_t>(m) * Nout + col0;
+    if (lim >= 32 && (Nout & 7) == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src) + q);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                r[8 * q + 2 * t] = __uint_as_float(w[t] << 16);
+                r[8 * q + 2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < lim) r[j] = __bfloat162float(src[j]);
+    }
+}
+
+// Final store of one output element; the in-place residual epilogue first
+// adds the value already there.
+__device__ __forceinline__ void store_out(__nv_bfloat16* o, int epi, float v)
+{
+    if (epi == MX_EPI_RESIDUAL) v += __bfloat162float(*o);
+    *o = __float2bfloat16_rn(v);
+}
+
 // Stores one warp's 32 x 32 chunk of bf16 results (row = lane, 16 packed
 // pairs per lane) through `buf`, 2 KB of the warp's own shared memory.  Each
 // lane parks its row's 64 bytes there, 16-byte pieces XOR-swizzled by row

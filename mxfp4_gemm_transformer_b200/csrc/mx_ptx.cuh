@@ -193,6 +193,19 @@ __device__ __forceinline__ void mma_mx(uint32_t d, uint64_t adesc, uint64_t bdes
         : "memory");
 }
 
+// D(tmem) (+)= A(smem) x B(smem), both packed e2m1 (K = 64 per instruction),
+// two E8M0 scales per row per instruction (kind::mxf4, 32-element blocks).
+__device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
 // D(tmem) (+)= A(smem) x B(smem) without block scales (kind::f8f6f4).
 __device__ __forceinline__ void mma_f8(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate)

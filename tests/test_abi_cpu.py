@@ -94,6 +94,36 @@ def test_quant_validation(lib):
     assert lib.mx_quant_weight(P[0], 64, 64, P[1], P[2], 3, None) == mxg.MX_ERR_FORMAT
 
 
+def test_residual_epilogue_validation(lib):
+    # the residual epilogue takes a bias or none
+    assert gemm(lib, epi=4, a=None) == mxg.MX_ERR_NULL
+    assert gemm(lib, epi=4, out=P[5] + 4) == mxg.MX_ERR_ALIGN
+
+
+def test_add_rms_quant_validation(lib):
+    f = lib.mx_add_rms_quant
+    ok = dict(x=P[0], r=P[1], w=P[2], eps=1e-6, M=4, K=64, y=P[3], c=P[4], s=P[5])
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["x"], a["r"], a["w"], a["eps"], a["M"], a["K"], a["y"], a["c"], a["s"], None)
+    assert call(x=None) == mxg.MX_ERR_NULL
+    assert call(r=None) == mxg.MX_ERR_NULL
+    assert call(w=None) == mxg.MX_ERR_NULL
+    assert call(c=None) == mxg.MX_ERR_NULL
+    assert call(s=None) == mxg.MX_ERR_NULL
+    assert call(K=48) == mxg.MX_ERR_SHAPE
+    assert call(K=16416) == mxg.MX_ERR_SHAPE
+    assert call(M=0) == mxg.MX_ERR_SHAPE
+    assert call(eps=-1.0) == mxg.MX_ERR_SHAPE
+    assert call(eps=float("nan")) == mxg.MX_ERR_SHAPE
+    assert call(x=P[0] + 8) == mxg.MX_ERR_ALIGN
+    assert call(y=P[3] + 2) == mxg.MX_ERR_ALIGN
+    if not torch.cuda.is_available():
+        assert call(y=None) in (mxg.MX_ERR_CUDA, mxg.MX_ERR_ARCH)  # y_out is optional
+
+
 def test_workspace_size(lib):
     assert lib.mx_gemm_workspace_size(16, 256, 512, 0, 0, 1) >= 4
 

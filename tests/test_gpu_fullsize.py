@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 E8, E2, F32 = 0, 1, 2
 NONE, BIAS, GELU, SWIGLU = 0, 1, 2, 3
 
-# (name, M, N, K, b_fmt, epi, seed, with_bias); seeds as in bench.py
+# (name, M, N, K, b_fmt, epi, seed, with_bias[, a_fmt]); seeds as in bench.py
 WORKLOADS = [
     ("decode q_a+kv M=1", 1, 2048, 7168, E8, NONE, 1, False),
     ("decode q_a+kv M=8", 8, 2048, 7168, E8, NONE, 1, False),
@@ -32,6 +32,9 @@ WORKLOADS = [
     ("W4A8 gate_up SwiGLU M=16", 16, 34816, 5120, E2, SWIGLU, 3, False),
     ("W4A8 gate_up SwiGLU M=4096", 4096, 34816, 5120, E2, SWIGLU, 3, False),
     ("fp8 lm_head", 16, 248320, 5120, F32, NONE, 4, False),
+    ("W4A8 down projection M=16", 16, 5120, 17408, E2, NONE, 5, False),
+    ("W4A8 down projection M=4096", 4096, 5120, 17408, E2, NONE, 5, False),
+    ("W4A4 gate_up SwiGLU M=4096", 4096, 34816, 5120, E2, SWIGLU, 3, False, 3),
 ]
 
 
@@ -68,9 +71,10 @@ def sample_blocks(nout, tile_n, rng):
     return np.array(sorted(blocks), np.int64)
 
 
-@pytest.mark.parametrize("name,M,N,K,b_fmt,epi,seed,with_bias", WORKLOADS, ids=[w[0] for w in WORKLOADS])
-def test_full_size_sampled(mx, name, M, N, K, b_fmt, epi, seed, with_bias):
-    a_fmt = 1 if b_fmt == F32 else 0
+@pytest.mark.parametrize("name,M,N,K,b_fmt,epi,seed,with_bias,a_fmt",
+                         [w if len(w) == 9 else w + (1 if w[4] == F32 else 0,) for w in WORKLOADS],
+                         ids=[w[0] for w in WORKLOADS])
+def test_full_size_sampled(mx, name, M, N, K, b_fmt, epi, seed, with_bias, a_fmt):
     dev = "cuda"
     # ---- GPU: the whole problem, as the bench runs it
     w = synth.bf16_matrix(seed + 1, N, K, synth.W_SIGMA, device=dev)
