@@ -834,6 +834,74 @@ def run_profile_only(args):
         sys.exit(3)
 
 
+# routed-expert gate_up of a mixture-of-experts layer, W4A8 (the DeepSeek-V4
+# mono runner page's w13 layout: [experts, 2 inter, hidden / 2] e2m1 with 1x32
+# E8M0 scales), hidden 7168, 2 x inter = 1024, SwiGLU; the tokens routed to
+# 8 local experts, unevenly, one expert empty
+MOE_COUNTS = (448, 384, 320, 288, 256, 192, 160, 0)
+MOE_N, MOE_K = 1024, 7168
+
+
+def moe_grouped_workload(mx, stream, pk, seed=6):
+    """One mx_gemm_grouped launch over every expert against one mx_gemm launch
+    per non-empty expert, graphs of back-to-back launches over rotating
+    weight copies (> 2x L2)."""
+    import synth
+    E, N, K = len(MOE_COUNTS), MOE_N, MOE_K
+    offsets = [0]
+    for c in MOE_COUNTS:
+        offsets.append(offsets[-1] + c)
+    M = offsets[-1]
+    x = synth.bf16_matrix(seed, M, K, synth.X_SIGMA, device="cuda")
+    ac, asc = mx.act_buffers(M, K)
+    mx.mx_quant_act(x, ac, asc)
+    wc = torch.empty(E * N, K // 2, dtype=torch.uint8, device="cuda")
+    wsc = torch.empty(E * N, K // 32, dtype=torch.uint8, device="cuda")
+    for e in range(E):
+        w = synth.bf16_matrix(seed + 10 + e, N, K, synth.W_SIGMA, device="cuda")
+        mx.mx_quant_weight(w, wc[e * N:(e + 1) * N], wsc[e * N:(e + 1) * N], mx.MX_B_E2M1_E8M0_1X32)
+    torch.cuda.synchronize()
+    w_bytes = wc.numel() + wsc.numel()
+    copies = min(32, max(1, math.ceil(2 * L2_BYTES / w_bytes)))
+    weights = [(wc, wsc)] + [(wc.clone(), wsc.clone()) for _ in range(copies - 1)]
+    out = mx.out_buffer(M, N, mx.MX_EPI_SWIGLU)
+    ws = mx.workspace()
+    launches = max(copies, 8)
+
+    def grouped_body():
+        for i in range(launches):
+            b, sb = weights[i % copies]
+            mx.mx_gemm_grouped(ac, asc, 0, b, sb, 1, None, mx.MX_EPI_SWIGLU, out, offsets, N, K, ws, stream=stream)
+
+    def per_expert_body():
+        for i in range(launches):
+            b, sb = weights[i % copies]
+            for e in range(E):
+                r0, r1 = offsets[e], offsets[e + 1]
+                if r1 == r0:
+                    continue
+                mx.mx_gemm(ac[r0:r1], asc[r0:r1], 0, b[e * N:(e + 1) * N], sb[e * N:(e + 1) * N], 1, None,
+                           mx.MX_EPI_SWIGLU, out[r0:r1], r1 - r0, N, K, ws, stream=stream)
+    with torch.cuda.stream(stream):
+        grouped_body()
+        per_expert_body()
+    stream.synchronize()
+    assert mx.mx_workspace_status(ws) == mx.MX_OK
+    tg = launch_time(capture(stream, grouped_body), launches, stream, 0.3)
+    tp = launch_time(capture(stream, per_expert_body), launches, stream, 0.3)
+    flops = 2.0 * M * N * K
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    ach = flops / tg / 1e12
+    return {"workload": f"grouped MoE gate_up W4A8 + SwiGLU: {E} experts, rows {list(MOE_COUNTS)}, "
+                        f"N={N} (2 x inter), K={K}",
+            "gemm_us": round(tg * 1e6, 3), "per_expert_launches_us": round(tp * 1e6, 3),
+            "tflops": round(ach, 2),
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4), "traffic": None,
+                         "peak_note": f"fp8 = 2 x {pk['source']} bf16 burst"},
+            "rotating_copies": copies}
+
+
 def extra_workloads(mx, stream, pk):
     """The other workloads, each GEMM timed alone (graph of back-to-back
     launches over rotating weights) against its roofline."""
@@ -870,6 +938,12 @@ def extra_workloads(mx, stream, pk):
             torch.cuda.empty_cache()
         except Exception as e:  # report, keep going
             res.append({"workload": name, "error": repr(e)[:300]})
+    log("workload: grouped MoE gate_up")
+    try:
+        res.append(moe_grouped_workload(mx, stream, pk))
+    except Exception as e:
+        res.append({"workload": "grouped MoE gate_up", "error": repr(e)[:300]})
+    torch.cuda.empty_cache()
     return res
 
 

@@ -261,6 +261,39 @@ MX_API mx_status mx_gemm(const void* a_codes, const void* a_scales, mx_a_fmt a_f
                   int K, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * mx_gemm_grouped -- `groups` independent GEMMs that share N, K, formats and
+ * epilogue in one launch: the routed experts of a mixture-of-experts layer
+ * (vLLM DeepSeek-V4 mono runner page, MonoLayerWeights: w13 [experts,
+ * 2 inter, hidden / 2] and w2 [experts, hidden, inter / 2] fp4x2 with their
+ * 1 x 32 E8M0 scales [experts * rows, hidden / 32]).  The tokens come sorted
+ * by group: activation rows offsets[g] .. offsets[g + 1] - 1 go through group
+ * g's weights and bias, and the result lands in the same rows of out.
+ *
+ *   a_codes, a_scales  [M, K] activations of every group, M = offsets[groups];
+ *                      MX_A_E4M3_E8M0_1X32 or MX_A_E2M1_E8M0_1X32 (W4A4).
+ *   b_codes, b_scales  the groups' weights back to back: codes [groups * N,
+ *                      K] (e4m3) or [groups * N, K/2] (e2m1), scales as the
+ *                      B format lays out groups * N rows ([groups * N / 32,
+ *                      K/32] for 32 x 32 blocks, [groups * N, K/32] for 1 x 32).
+ *   bias               fp32 [groups, N] or NULL (rules of mx_gemm).
+ *   epi                any mx_epi but MX_EPI_SWIGLU_MXQ.
+ *   out                [M, N] bf16 ([M, N/2] for SWIGLU).
+ *   offsets            HOST array of groups + 1 ints: 0 = offsets[0] <=
+ *                      offsets[1] <= ... ; a group may be empty.
+ *   workspace          as mx_gemm (the 256-byte minimum is enough).
+ * Requires 1 <= groups <= 256; shapes, alignment and format pairs as mx_gemm
+ * (F32_ROW and bf16 activations are not taken).  The groups' tiles share one
+ * persistent launch of the tile kernel, whatever the rows per group, so
+ * small groups do not each pay a launch.  M = 0 (every group empty) returns
+ * MX_OK and launches nothing.
+ */
+MX_API mx_status mx_gemm_grouped(const void* a_codes, const void* a_scales, mx_a_fmt a_fmt, const void* b_codes,
+                                 const void* b_scales, mx_b_fmt b_fmt, const float* bias, mx_epi epi, void* out,
+                                 int groups, const int* offsets, int N, int K, void* workspace, size_t ws_bytes,
+                                 void* stream);
+#define MX_MAX_GROUPS 256
+
+/*
  * mx_gemm_noalloc -- mx_gemm for callers that cannot allocate device memory.
  * The pages have no counterpart to this call; it exists for users of this
  * library who cannot hand mx_gemm a workspace: code running while a stream is

@@ -24,11 +24,12 @@ MX_EPI_SWIGLU_MXQ = 5
 
 MX_LAUNCH_PDL, MX_LAUNCH_PREFETCH_WEIGHTS, MX_LAUNCH_DETERMINISTIC = 1, 2, 4
 MX_TUNE_BM_PAIR = 2  # mx_set_tuning block_m: 256 x 240 tiles over CTA pairs
+MX_MAX_GROUPS = 256  # groups one mx_gemm_grouped call takes
 
 MX_OK, MX_ERR_NULL, MX_ERR_SHAPE, MX_ERR_ALIGN, MX_ERR_FORMAT = 0, 1, 2, 3, 4
 MX_ERR_WORKSPACE, MX_ERR_ARCH, MX_ERR_CUDA, MX_ERR_TIMEOUT = 5, 6, 7, 8
 
-EXPORTS = ["mx_quant_act", "mx_quant_weight", "mx_add_rms_quant", "mx_gemm_workspace_size", "mx_gemm", "mx_status_string",
+EXPORTS = ["mx_quant_act", "mx_quant_weight", "mx_add_rms_quant", "mx_gemm_grouped", "mx_gemm_workspace_size", "mx_gemm", "mx_status_string",
            "mx_workspace_status", "mx_debug_watchdog", "mx_set_tuning", "mx_gemm_plan", "mx_gemm_noalloc",
            "mx_debug_set_timeline", "mx_set_launch_flags", "mx_set_decode_tuning", "mx_gemm_plan_info"]
 
@@ -75,6 +76,7 @@ def load(path: str | None = None):
         "mx_set_tuning": (None, [I, I, I, I]),
         "mx_gemm_plan": (I, [I, I, I, I, I, I, IP, IP, IP, IP]),
         "mx_gemm_noalloc": (I, [P, P, I, P, P, I, P, I, P, I, I, I, P]),
+        "mx_gemm_grouped": (I, [P, P, I, P, P, I, P, I, P, I, IP, I, I, P, S, P]),
         "mx_debug_set_timeline": (None, [P, S]),
         "mx_set_launch_flags": (None, [U]),
         "mx_set_decode_tuning": (None, [I, I, I, I, I, I]),
@@ -147,6 +149,21 @@ def mx_gemm(a_codes, a_scales, a_fmt, b_codes, b_scales, b_fmt, bias, epi, out, 
         ws_bytes = workspace.numel() * workspace.element_size()
     _check(load().mx_gemm(_p(a_codes), _p(a_scales), a_fmt, _p(b_codes), _p(b_scales), b_fmt, _p(bias), epi,
                           _p(out), M, N, K, _p(workspace), ws_bytes, _stream(stream)), "mx_gemm")
+
+
+def mx_gemm_grouped(a_codes, a_scales, a_fmt, b_codes, b_scales, b_fmt, bias, epi, out, offsets, N, K, workspace,
+                    ws_bytes=None, stream=None):
+    """Grouped GEMM over routed experts: rows offsets[g] .. offsets[g+1]-1 of
+    the activations through group g's weights (b_codes / b_scales hold every
+    group's rows back to back, bias is [groups, N] or None); offsets is a host
+    sequence of groups + 1 ints."""
+    offs = [int(o) for o in offsets]
+    arr = (ctypes.c_int * len(offs))(*offs)
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().mx_gemm_grouped(_p(a_codes), _p(a_scales), a_fmt, _p(b_codes), _p(b_scales), b_fmt, _p(bias), epi,
+                                  _p(out), len(offs) - 1, arr, N, K, _p(workspace), ws_bytes, _stream(stream)),
+           "mx_gemm_grouped")
 
 
 def mx_gemm_noalloc(a_codes, a_scales, a_fmt, b_codes, b_scales, b_fmt, bias, epi, out, M, N, K, stream=None):

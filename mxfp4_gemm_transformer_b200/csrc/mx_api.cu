@@ -100,6 +100,35 @@ const char* mx_status_string(mx_status s)
     return "unknown mx_status";
 }
 
+mx_status mx_gemm_grouped(const void* a_codes, const void* a_scales, mx_a_fmt a_fmt, const void* b_codes,
+                          const void* b_scales, mx_b_fmt b_fmt, const float* bias, mx_epi epi, void* out, int groups,
+                          const int* offsets, int N, int K, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!offsets) return MX_ERR_NULL;
+    if (groups < 1 || groups > kMaxGroups || offsets[0] != 0) return MX_ERR_SHAPE;
+    for (int g = 0; g < groups; ++g)
+        if (offsets[g + 1] < offsets[g]) return MX_ERR_SHAPE;
+    const int M = offsets[groups];
+    if (a_fmt != MX_A_E4M3_E8M0_1X32 && a_fmt != MX_A_E2M1_E8M0_1X32) return MX_ERR_FORMAT;
+    if (epi == MX_EPI_SWIGLU_MXQ) return MX_ERR_FORMAT;
+    // shapes and formats as mx_gemm (one row stands in when every group is empty)
+    mx_status s = validate_gemm(a_codes, a_scales, a_fmt, b_codes, b_scales, b_fmt, bias, epi, out, M > 0 ? M : 1, N,
+                                K);
+    if (s != MX_OK) return s;
+    if (static_cast<long long>(groups) * N > (1LL << 31) - 1) return MX_ERR_SHAPE;
+    if (!workspace || ws_bytes < kWorkspaceBytes) return MX_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return MX_ERR_ALIGN;
+    DeviceInfo dev;
+    s = arch_ok(&dev);
+    if (s != MX_OK) return s;
+    if (M == 0) return MX_OK;  // no rows in any group: nothing to compute
+    GemmProblem pb{a_codes, a_scales, a_fmt, b_codes, b_scales, b_fmt, bias, epi, out, M, N, K,
+                   static_cast<unsigned*>(workspace), groups, offsets};
+    GemmPlan plan;
+    if (plan_gemm_grouped(pb, dev, &plan) != cudaSuccess) return MX_ERR_CUDA;
+    return from_cuda(launch_gemm(pb, plan, static_cast<cudaStream_t>(stream)));
+}
+
 mx_status mx_quant_act(const void* x, int M, int K, void* codes, void* scales, mx_a_fmt fmt, void* stream)
 {
     if (!x || !codes || !scales) return MX_ERR_NULL;

@@ -68,7 +68,45 @@ struct GemmArgs {
     int b_fmt, epi, n_half;
     uint32_t idesc;
     uint32_t tx_bytes;
+    // Grouped launch (routed experts), groups > 0: group g takes activation
+    // rows g_row[g] .. g_row[g+1]-1 through weight rows g*N .. g*N+N-1 (and
+    // bias g*N ..), and owns units g_unit[g] .. g_unit[g+1]-1 of the walk, its
+    // M tiles times tiles_n; b_rows = every group's weight rows (load bound).
+    int groups, b_rows;
+    int g_row[kMaxGroups + 1];
+    int g_unit[kMaxGroups + 1];
 };
+
+static_assert(sizeof(GemmArgs) <= 4096, "kernel parameters must fit the 4 KB parameter space");
+
+// Where one output tile lies: activation rows m0 .. m_end-1 (m_end bounds the
+// rows of its group), weight rows from b0, column tile tn, the group's bias.
+struct TileXY {
+    int m0, m_end, b0, tn;
+    const float* bias;
+};
+
+__device__ __forceinline__ TileXY tile_xy(const GemmArgs& p, int tile, int bm)
+{
+    if (p.groups == 0) {
+        const int tm = tile % p.tiles_m;
+        return TileXY{tm * bm, p.M, 0, tile / p.tiles_m, p.bias};
+    }
+    // the group whose units hold this tile: the last g with g_unit[g] <= tile
+    // (empty groups own no units, so a run of equal starts resolves to the
+    // group after it)
+    int lo = 0, hi = p.groups;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (p.g_unit[mid] <= tile) lo = mid;
+        else hi = mid;
+    }
+    const int r0 = p.g_row[lo], r1 = p.g_row[lo + 1];
+    const int tiles_m = (r1 - r0 + bm - 1) / bm;
+    const int local = tile - p.g_unit[lo];
+    return TileXY{r0 + (local % tiles_m) * bm, r1, lo * p.N, local / tiles_m,
+                  p.bias ? p.bias + static_cast<size_t>(lo) * p.N : nullptr};
+}
 
 // AR = rows of the activation tile loaded per stage:
 //   64   decode (M <= 64): the MMA still reads 128 rows; accumulator rows >= 64
@@ -301,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             int pre = 0;
             if (p.prefetch_w && u_first < p.units) {
                 const int tile = u_first / p.splits, split = u_first % p.splits;
-                const int tn = tile / p.tiles_m;
+                const TileXY t = tile_xy(p, tile, C::BM);
                 const int kb0 = split * p.num_kb / p.splits, kb1 = (split + 1) * p.num_kb / p.splits;
                 pre = min(C::STAGES, kb1 - kb0);
                 for (int i = 0; i < pre; ++i) {
@@ -309,18 +347,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     mbar_arrive_expect_tx(&full[i], p.tx_bytes);
                     uint8_t* sB = ring + i * C::STAGE_BYTES + C::A_BYTES;
                     if (SWIGLU) {
-                        tma_load_2d(sB, &p.tmB, &full[i], kb * C::BK, tn * (BN / 2), pol_b);
-                        tma_load_2d(sB + (BN / 2) * C::BK, &p.tmB, &full[i], kb * C::BK, p.n_half + tn * (BN / 2),
-                                    pol_b);
+                        tma_load_2d(sB, &p.tmB, &full[i], kb * C::BK, t.b0 + t.tn * (BN / 2), pol_b);
+                        tma_load_2d(sB + (BN / 2) * C::BK, &p.tmB, &full[i], kb * C::BK,
+                                    t.b0 + p.n_half + t.tn * (BN / 2), pol_b);
                     } else {
-                        tma_load_2d(sB, &p.tmB, &full[i], kb * C::BK, tn * BN, pol_b);
+                        tma_load_2d(sB, &p.tmB, &full[i], kb * C::BK, t.b0 + t.tn * BN, pol_b);
                     }
                 }
             }
             pdl_wait();
             for (int u = u_first; u < p.units; u += u_step) {
                 const int tile = u / p.splits, split = u % p.splits;
-                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                const TileXY t = tile_xy(p, tile, C::BM);
                 const int kb0 = split * p.num_kb / p.splits, kb1 = (split + 1) * p.num_kb / p.splits;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     uint8_t* sA = ring + stage * C::STAGE_BYTES;
@@ -328,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     if (pre > 0) {
                         // weights already requested; add the activation tile
                         --pre;
-                        tma_load_2d(sA, &p.tmA, &full[stage], kb * C::BK, tm * C::BM, pol_a);
+                        tma_load_2d(sA, &p.tmA, &full[stage], kb * C::BK, t.m0, pol_a);
                         if (u == u_first && kb == kb0) stamp(p, kStampFirstTma);
                         if (++stage == C::STAGES) {
                             stage = 0;
@@ -338,15 +376,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     }
                     if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.status)) goto producer_done;
                     mbar_arrive_expect_tx(&full[stage], p.tx_bytes);
-                    tma_load_2d(sA, &p.tmA, &full[stage], kb * C::BK, tm * C::BM, pol_a);
+                    tma_load_2d(sA, &p.tmA, &full[stage], kb * C::BK, t.m0, pol_a);
                     if (u == u_first && kb == kb0) stamp(p, kStampFirstTma);
                     stamp_stage(p, 0, dbg_i++);
                     if (SWIGLU) {
-                        tma_load_2d(sB, &p.tmB, &full[stage], kb * C::BK, tn * (BN / 2), pol_b);
+                        tma_load_2d(sB, &p.tmB, &full[stage], kb * C::BK, t.b0 + t.tn * (BN / 2), pol_b);
                         tma_load_2d(sB + (BN / 2) * C::BK, &p.tmB, &full[stage], kb * C::BK,
-                                    p.n_half + tn * (BN / 2), pol_b);
+                                    t.b0 + p.n_half + t.tn * (BN / 2), pol_b);
                     } else {
-                        tma_load_2d(sB, &p.tmB, &full[stage], kb * C::BK, tn * BN, pol_b);
+                        tma_load_2d(sB, &p.tmB, &full[stage], kb * C::BK, t.b0 + t.tn * BN, pol_b);
                     }
                     if (++stage == C::STAGES) {
                         stage = 0;
@@ -447,30 +485,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             int dbg_i = 0;
             const int KB = p.KB;
             const bool vec4 = (KB & 3) == 0;
-            auto issue_a = [&](uint8_t* sf, int tm, int k4) {
+            auto issue_a = [&](uint8_t* sf, int m0, int k4) {
 #pragma unroll
                 for (int rb = 0; rb < C::MB; ++rb) {
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
-                        const int m = tm * C::BM + rb * 128 + lane + 32 * g;
+                        const int m = m0 + rb * 128 + lane + 32 * g;
                         const bool ok = m < p.M;
                         const uint8_t* src = p.sa + static_cast<size_t>(ok ? m : 0) * KB + k4;
                         cp_async_4(sf + 512 * rb + lane * 16 + g * 4, src, ok ? 4u : 0u);
                     }
                 }
             };
-            auto b_row = [&](int r, int tn) {
-                if (SWIGLU) return (r < BN / 2) ? tn * (BN / 2) + r : p.n_half + tn * (BN / 2) + (r - BN / 2);
-                return tn * BN + r;
+            auto b_row = [&](int r, const TileXY& t) {
+                if (SWIGLU)
+                    return t.b0 + ((r < BN / 2) ? t.tn * (BN / 2) + r : p.n_half + t.tn * (BN / 2) + (r - BN / 2));
+                return t.b0 + t.tn * BN + r;
             };
-            auto issue_b = [&](uint8_t* sf, int tn, int k4) {
+            auto issue_b = [&](uint8_t* sf, const TileXY& t, int k4) {
 #pragma unroll
                 for (int j = 0; j < C::SFB_CHUNKS; ++j) {
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         const int r = 128 * j + lane + 32 * g;  // row within the B tile
-                        const int n = b_row(r, tn);
-                        const bool ok = r < BN && n < p.N;
+                        const int n = b_row(r, t);
+                        const bool ok = r < BN && n < p.b_rows;
                         const int nn = ok ? n : 0;
                         const uint8_t* src = (p.b_fmt == MX_B_E4M3_E8M0_32X32)
                                                  ? p.sb + static_cast<size_t>(nn >> 5) * KB + k4
@@ -484,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             int pre = 0;
             if (vec4 && p.prefetch_w && u_first < p.units) {
                 const int tile = u_first / p.splits, split = u_first % p.splits;
-                const int tn = tile / p.tiles_m;
+                const TileXY t = tile_xy(p, tile, C::BM);
                 const int kb0 = split * p.num_kb / p.splits, kb1 = (split + 1) * p.num_kb / p.splits;
                 pre = min(C::STAGES, kb1 - kb0);
                 for (int i = 0; i < pre; ++i) {
@@ -492,13 +531,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     const int kbase = (kb0 + i) * (C::KPS / 32);
 #pragma unroll
                     for (int c = 0; c < (F4 ? 2 : 1); ++c)
-                        if (kbase + 4 * c < KB) issue_b(sf + c * C::SF_CHUNK, tn, kbase + 4 * c);
+                        if (kbase + 4 * c < KB) issue_b(sf + c * C::SF_CHUNK, t, kbase + 4 * c);
                 }
             }
             pdl_wait();
             for (int u = u_first; u < p.units; u += u_step) {
                 const int tile = u / p.splits, split = u % p.splits;
-                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                const TileXY t = tile_xy(p, tile, C::BM);
                 const int kb0 = split * p.num_kb / p.splits, kb1 = (split + 1) * p.num_kb / p.splits;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     uint8_t* sf = ring + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
@@ -507,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                         --pre;
 #pragma unroll
                         for (int c = 0; c < (F4 ? 2 : 1); ++c)
-                            if (k4 + 4 * c < KB) issue_a(sf + c * C::SF_CHUNK, tm, k4 + 4 * c);
+                            if (k4 + 4 * c < KB) issue_a(sf + c * C::SF_CHUNK, t.m0, k4 + 4 * c);
                         cp_async_arrive_noinc(&full[stage]);
                     } else {
                         if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.status)) goto sf_done;
@@ -517,13 +556,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 #pragma unroll
                             for (int c = 0; c < 2; ++c)
                                 if (k4 + 4 * c < KB) {
-                                    issue_a(sf + c * C::SF_CHUNK, tm, k4 + 4 * c);
-                                    issue_b(sf + c * C::SF_CHUNK, tn, k4 + 4 * c);
+                                    issue_a(sf + c * C::SF_CHUNK, t.m0, k4 + 4 * c);
+                                    issue_b(sf + c * C::SF_CHUNK, t, k4 + 4 * c);
                                 }
                             cp_async_arrive_noinc(&full[stage]);
                         } else if (vec4) {
-                            issue_a(sf, tm, k4);
-                            issue_b(sf, tn, k4);
+                            issue_a(sf, t.m0, k4);
+                            issue_b(sf, t, k4);
                             cp_async_arrive_noinc(&full[stage]);
                             if (lane == 0) stamp_stage(p, 3, dbg_i);
                             ++dbg_i;
@@ -533,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                             for (int rb = 0; rb < C::MB; ++rb) {
 #pragma unroll
                                 for (int g = 0; g < 4; ++g) {
-                                    const int m = tm * C::BM + rb * 128 + lane + 32 * g;
+                                    const int m = t.m0 + rb * 128 + lane + 32 * g;
                                     uint32_t w = 0;
                                     if (m < p.M) {
                                         const uint8_t* src = p.sa + static_cast<size_t>(m) * KB + k4;
@@ -550,9 +589,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 #pragma unroll
                                 for (int g = 0; g < 4; ++g) {
                                     const int r = 128 * j + lane + 32 * g;
-                                    const int n = b_row(r, tn);
+                                    const int n = b_row(r, t);
                                     uint32_t w = 0;
-                                    if (r < BN && n < p.N) {
+                                    if (r < BN && n < p.b_rows) {
                                         const uint8_t* src = (p.b_fmt == MX_B_E4M3_E8M0_32X32)
                                                                  ? p.sb + static_cast<size_t>(n >> 5) * KB + k4
                                                                  : p.sb + static_cast<size_t>(n) * KB + k4;
@@ -730,23 +769,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 continue;
             }
             // stage this tile's per-column parameters in shared memory
-            const int n_base = tn * C::OUT_COLS;
+            const TileXY t = tile_xy(p, tile, C::BM);
+            const int n_base = t.tn * C::OUT_COLS;
             for (int i = et; i < C::OUT_COLS; i += kEpiThreads) {
                 const int n = n_base + i;
                 const bool ok = n < p.Nout;
-                colp[i] = (ok && p.bias) ? __ldcg(p.bias + n) : 0.f;
-                colp[256 + i] = (SWIGLU && ok && p.bias) ? __ldcg(p.bias + n + p.n_half) : 0.f;
+                colp[i] = (ok && t.bias) ? __ldcg(t.bias + n) : 0.f;
+                colp[256 + i] = (SWIGLU && ok && t.bias) ? __ldcg(t.bias + n + p.n_half) : 0.f;
                 colp[512 + i] = (f32row && ok) ? __ldcg(p.swb + n) : 1.f;
                 colp[768 + i] = (SWIGLU && f32row && ok) ? __ldcg(p.swb + n + p.n_half) : 1.f;
             }
             named_bar_sync(1, kEpiThreads);
 #pragma unroll 1
             for (int rb = 0; rb < C::MB; ++rb) {
-                const int m = tm * C::BM + rb * 128 + row;
-                if (tm * C::BM + rb * 128 + q * 32 >= p.M) continue;  // warp-uniform: no valid row
+                const int m = t.m0 + rb * 128 + row;
+                if (t.m0 + rb * 128 + q * 32 >= t.m_end) continue;  // warp-uniform: no valid row
                 const uint32_t taddr =
                     tmem + acc * C::ACC_STRIDE + rb * C::RB_STRIDE + (static_cast<uint32_t>(q * 32) << 16);
-                const bool row_ok = m < p.M;
+                const bool row_ok = m < t.m_end;
                 const float sx = (f32row && row_ok) ? __ldcg(p.sxa + m) : 1.f;
                 __nv_bfloat16* out_row = p.out + static_cast<size_t>(row_ok ? m : 0) * p.Nout + n_base;
 #pragma unroll 1
@@ -767,8 +807,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                         else epi_chunk<MX_EPI_BIAS, false, false>(g, h, sx, colp, c, pk);
                     } else if (p.epi == MX_EPI_RESIDUAL) {
                         float res[32];
-                        load_row32_bf16(p.out, p.Nout, p.M, m, n_base + c, min(min(32, C::OUT_COLS - c), p.Nout - (n_base + c)),
-                                        res);
+                        load_row32_bf16(p.out, p.Nout, t.m_end, m, n_base + c,
+                                        min(min(32, C::OUT_COLS - c), p.Nout - (n_base + c)), res);
                         if (f32row) epi_chunk_residual<true>(g, sx, colp, c, res, pk);
                         else epi_chunk_residual<false>(g, sx, colp, c, res, pk);
                     } else {
@@ -778,8 +818,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     const int cw = min(32, C::OUT_COLS - c);  // columns of this chunk in the tile
                     const int n_left = p.Nout - (n_base + c);
                     if (C::STAGING_BYTES > 0) {
-                        store_chunk_staged(staging + (warp - 4) * 2048, pk, lane, p.out, p.Nout, p.M,
-                                           tm * C::BM + rb * 128 + q * 32, n_base + c, min(cw, n_left));
+                        store_chunk_staged(staging + (warp - 4) * 2048, pk, lane, p.out, p.Nout, t.m_end,
+                                           t.m0 + rb * 128 + q * 32, n_base + c, min(cw, n_left));
                     } else if (row_ok) {
                         if (cw == 32 && n_left >= 32 && (p.Nout & 7) == 0) {
                             uint4* d4 = reinterpret_cast<uint4*>(out_row + c);
@@ -1314,8 +1354,16 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
         const int per_sm = g_dec_per_sm > 0 ? g_dec_per_sm : 2;
         int split = g_dec_split;
         if (split == kDecStreamK && det) split = kDecAuto;
-        const int cluster = g_dec_cluster > 0 ? g_dec_cluster
-                                              : std::min(8, (short_launch ? sms : 2 * sms) / std::max(1, tiles_d));
+        int cluster = g_dec_cluster > 0 ? g_dec_cluster
+                                        : std::min(8, (short_launch ? sms : 2 * sms) / std::max(1, tiles_d));
+        // A short launch whose CTAs would each stream many K blocks (the W4A8
+        // down projection at M = 16: 40 tiles x 136 K blocks) fills two CTAs
+        // per SM instead, in clusters of at most 6 (measured there: 15.2 us
+        // against 23.8 us for clusters of 3, one CTA per SM; clusters of 7 at
+        // two per SM ran at 25 us).
+        const int num_kb_d = (pb.K + 127) / 128;
+        if (g_dec_cluster == 0 && short_launch && num_kb_d > 16 * cluster)
+            cluster = std::min(6, 2 * sms / std::max(1, tiles_d));
         GemmPlan dp;
         if ((split == kDecAuto || split == kDecCluster) && tiles_d * cluster <= 2 * sms &&
             plan_decode(pb, kDecCluster, grid, cluster, per_sm, sms, &dp)) {
@@ -1460,6 +1508,41 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
     return cudaSuccess;
 }
 
+// Grouped problems run on the tile kernel: tiles of 128 activation rows of
+// one group by 240 weight rows (the variant with two accumulators, so one
+// tile's epilogue overlaps the next tile's main loop), no K split, one
+// persistent CTA per SM.  mx_set_tuning may pick 128 / 256 columns (240 / 256
+// for W4A4) and cap the CTAs.
+cudaError_t plan_gemm_grouped(const GemmProblem& pb, const DeviceInfo& dev, GemmPlan* plan)
+{
+    const bool swiglu = epi_swiglu(pb.epi);
+    const int sc = pb.a_fmt == MX_A_E2M1_E8M0_1X32 ? 2 : 1;
+    int bn = 240;
+    if (g_tune_bn == 256 || (sc == 1 && g_tune_bn == 128)) bn = g_tune_bn;
+    const int oc = swiglu ? bn / 2 : bn;
+    const int tiles_n = ((swiglu ? pb.N / 2 : pb.N) + oc - 1) / oc;
+    long long units = 0;
+    for (int g = 0; g < pb.groups; ++g) units += (pb.offsets[g + 1] - pb.offsets[g] + 127) / 128 * tiles_n;
+    if (units > (1LL << 30)) return cudaErrorInvalidValue;
+    *plan = GemmPlan();
+    plan->kernel = 0;
+    plan->block_n = bn;
+    plan->a_rows = 128;
+    plan->block_m = 128;
+    plan->splits = 1;
+    plan->gsplit = 0;
+    plan->units = static_cast<int>(units);
+    plan->tiles = static_cast<int>(units);
+    int grid = static_cast<int>(std::min<long long>(units, dev.sms));
+    if (g_tune_ctas > 0) grid = std::min(grid, g_tune_ctas);
+    plan->grid_x = std::max(grid, 1);
+    plan->grid_y = 1;
+    plan->ws_bytes = kWorkspaceHeader;
+    plan->acc_bufs = dispatch(bn, 128, sc, swiglu, AccBufsOp{});
+    plan->stages = dispatch(bn, 128, sc, swiglu, StagesOp{});
+    return plan->acc_bufs > 0 ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_t st)
 {
     if (plan.act_quant == 2) {
@@ -1506,22 +1589,40 @@ cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_
     memset(&a, 0, sizeof(a));
     const bool f4 = pb.a_fmt == MX_A_E2M1_E8M0_1X32;  // W4A4, kind::mxf4
     const uint32_t b_rows = swiglu ? bn / 2 : bn;
+    // weight rows behind the map: every group's when the problems are grouped
+    const uint64_t nb = pb.groups > 0 ? static_cast<uint64_t>(pb.groups) * pb.N : static_cast<uint64_t>(pb.N);
     if (f4) {
         // both operands packed two per byte, loaded as plain bytes: a 128-byte
         // row of a stage holds 256 K elements
         if (!make_map(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.a_codes, pb.K / 2, pb.M, pb.K / 2, 128,
                       static_cast<uint32_t>(plan.a_rows)) ||
-            !make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.b_codes, pb.K / 2, pb.N, pb.K / 2, 128, b_rows))
+            !make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.b_codes, pb.K / 2, nb, pb.K / 2, 128, b_rows))
             return cudaErrorInvalidValue;
     } else if (!make_map(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.a_codes, pb.K, pb.M, pb.K, 128,
                          static_cast<uint32_t>(plan.a_rows))) {
         return cudaErrorInvalidValue;
     } else if (pb.b_fmt == MX_B_E2M1_E8M0_1X32) {
-        if (!make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, pb.b_codes, pb.K, pb.N, pb.K / 2, 128, b_rows))
+        if (!make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, pb.b_codes, pb.K, nb, pb.K / 2, 128, b_rows))
             return cudaErrorInvalidValue;
     } else {
-        if (!make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.b_codes, pb.K, pb.N, pb.K, 128, b_rows))
+        if (!make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.b_codes, pb.K, nb, pb.K, 128, b_rows))
             return cudaErrorInvalidValue;
+    }
+    a.b_rows = static_cast<int>(nb);
+    if (pb.groups > 0) {
+        // the group table: rows and first unit of every group (empty groups
+        // own no units); tiles are block_m rows of one group by out_cols
+        const int tiles_n = ((swiglu ? pb.N / 2 : pb.N) + out_cols - 1) / out_cols;
+        int unit = 0;
+        a.groups = pb.groups;
+        for (int g = 0; g < pb.groups; ++g) {
+            a.g_row[g] = pb.offsets[g];
+            a.g_unit[g] = unit;
+            unit += (pb.offsets[g + 1] - pb.offsets[g] + plan.block_m - 1) / plan.block_m * tiles_n;
+        }
+        a.g_row[pb.groups] = pb.offsets[pb.groups];
+        a.g_unit[pb.groups] = unit;
+        if (unit != plan.units) return cudaErrorInvalidValue;
     }
     a.sa = scaled ? static_cast<const uint8_t*>(pb.a_scales) : nullptr;
     a.sb = scaled ? static_cast<const uint8_t*>(pb.b_scales) : nullptr;
@@ -1547,7 +1648,7 @@ cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_
     a.Nout = swiglu ? pb.N / 2 : pb.N;
     a.KB = pb.K / 32;
     a.num_kb = f4 ? (pb.K + 255) / 256 : (pb.K + 127) / 128;
-    a.tiles_m = (pb.M + plan.block_m - 1) / plan.block_m;
+    a.tiles_m = pb.groups > 0 ? 1 : (pb.M + plan.block_m - 1) / plan.block_m;
     a.tiles_n = (a.Nout + out_cols - 1) / out_cols;
     a.splits = plan.splits;
     a.units = plan.units;

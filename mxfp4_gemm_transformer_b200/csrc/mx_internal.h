@@ -71,6 +71,10 @@ inline size_t act_quant_bytes(int M, int K)
     return codes + scales;
 }
 
+// Most groups one grouped launch takes (the group table travels in the
+// kernel's parameters).
+constexpr int kMaxGroups = 256;
+
 struct GemmProblem {
     const void* a_codes;
     const void* a_scales;
@@ -83,6 +87,10 @@ struct GemmProblem {
     void* out;
     int M, N, K;
     unsigned* status;
+    // grouped launch: `groups` problems sharing N, K, formats and epilogue;
+    // host offsets[0 .. groups] of their activation rows (M = offsets[groups])
+    int groups = 0;
+    const int* offsets = nullptr;
 };
 
 struct GemmPlan {
@@ -130,6 +138,8 @@ constexpr size_t kWorkspaceHeader = 256;
 // more are not considered).
 cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_bytes, GemmPlan* plan);
 cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_t st);
+// grouped problems (pb.groups > 0): the tile kernel over every group's tiles
+cudaError_t plan_gemm_grouped(const GemmProblem& pb, const DeviceInfo& dev, GemmPlan* plan);
 cudaError_t launch_watchdog_probe(unsigned* status, unsigned timeout_us, cudaStream_t st);
 
 void set_tuning(int block_n, int splits, int max_ctas, int block_m);

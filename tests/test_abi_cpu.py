@@ -124,6 +124,30 @@ def test_add_rms_quant_validation(lib):
         assert call(y=None) in (mxg.MX_ERR_CUDA, mxg.MX_ERR_ARCH)  # y_out is optional
 
 
+def test_grouped_validation(lib):
+    def call(offs, **kw):
+        a = dict(a=P[0], sa=P[1], af=0, b=P[2], sb=P[3], bf=1, bias=None, epi=0, out=P[5], N=256, K=512, ws=P[6],
+                 wsb=256)
+        a.update(kw)
+        arr = None if offs is None else (ctypes.c_int * len(offs))(*offs)
+        return lib.mx_gemm_grouped(a["a"], a["sa"], a["af"], a["b"], a["sb"], a["bf"], a["bias"], a["epi"], a["out"],
+                                   0 if offs is None else len(offs) - 1, arr, a["N"], a["K"], a["ws"], a["wsb"], None)
+    assert call(None) == mxg.MX_ERR_NULL
+    assert call([0]) == mxg.MX_ERR_SHAPE                      # no group
+    assert call([1, 4]) == mxg.MX_ERR_SHAPE                   # offsets start at 0
+    assert call([0, 5, 3]) == mxg.MX_ERR_SHAPE                # decreasing
+    assert call([0] * 258) == mxg.MX_ERR_SHAPE                # more than MX_MAX_GROUPS
+    assert call([0, 4], af=1, bf=2) == mxg.MX_ERR_FORMAT      # fp32-row formats are not grouped
+    assert call([0, 4], af=2) == mxg.MX_ERR_FORMAT            # nor bf16 activations
+    assert call([0, 4], epi=5) == mxg.MX_ERR_FORMAT           # nor the MX-code output
+    assert call([0, 4], epi=1) == mxg.MX_ERR_NULL             # BIAS needs a bias
+    assert call([0, 4], K=160) == mxg.MX_ERR_SHAPE            # e2m1 needs K % 128
+    assert call([0, 4], ws=None) == mxg.MX_ERR_WORKSPACE
+    assert call([0, 4], out=P[5] + 4) == mxg.MX_ERR_ALIGN
+    if not torch.cuda.is_available():
+        assert call([0, 4, 4]) in (mxg.MX_ERR_CUDA, mxg.MX_ERR_ARCH)
+
+
 def test_workspace_size(lib):
     assert lib.mx_gemm_workspace_size(16, 256, 512, 0, 0, 1) >= 4
 
