@@ -398,17 +398,25 @@ def kernel_timing(wl: Workload, M, stream, seconds=0.3):
     return tg, tq, tf
 
 
-KERNEL_SOURCES = ("mxfp4_gemm_transformer_b200/csrc/mx_gemm.cu", "mxfp4_gemm_transformer_b200/csrc/mx_decode.cu",
-                  "mxfp4_gemm_transformer_b200/csrc/mx_ptx.cuh", "mxfp4_gemm_transformer_b200/csrc/mx_internal.h",
-                  "mxfp4_gemm_transformer_b200/csrc/mx_kernel_common.cuh",
-                  "mxfp4_gemm_transformer_b200/csrc/mx_quant_common.cuh",
-                  "mxfp4_gemm_transformer_b200/csrc/mx_decode_common.cuh")
+# Sources each kernel family's code comes from: a traffic row in
+# profiles/traffic.md counts only while its family's sources hash to the value
+# recorded beside it.
+_CSRC = "mxfp4_gemm_transformer_b200/csrc/"
+KERNEL_FAMILIES = {
+    "decode": tuple(_CSRC + f for f in ("mx_decode.cu", "mx_decode_common.cuh", "mx_kernel_common.cuh",
+                                        "mx_quant_common.cuh", "mx_ptx.cuh", "mx_internal.h")),
+    "tile": tuple(_CSRC + f for f in ("mx_gemm.cu", "mx_kernel_common.cuh", "mx_ptx.cuh", "mx_internal.h")),
+}
+# the family of the kernel that runs each workload's GEMM on codes
+WORKLOAD_FAMILY = {"decode": "decode", "small": "decode", "gateup16": "decode", "gateup16_mxq": "decode",
+                   "down16": "decode", "lmhead": "decode", "mlp": "tile", "gateup4096": "tile",
+                   "down4096": "tile", "gateup4096_w4a4": "tile"}
 
 
-def kernel_hash() -> str:
+def kernel_hash(family: str) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_FAMILIES[family]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -419,12 +427,14 @@ def ncu_traffic():
     captured from the kernel sources as they are now (else nothing)."""
     out = {}
     try:
-        cur = kernel_hash()
+        cur = {fam: kernel_hash(fam) for fam in KERNEL_FAMILIES}
         with open(os.path.join(ROOT, "profiles", "traffic.md")) as f:
             for line in f:
                 cells = [c.strip() for c in line.strip().strip("|").split("|")]
-                if len(cells) == 4 and cells[1].isdigit() and cells[2].isdigit() and cells[3] == cur:
-                    out[(cells[0], int(cells[1]))] = int(cells[2])
+                if len(cells) == 4 and cells[1].isdigit() and cells[2].isdigit():
+                    fam = WORKLOAD_FAMILY.get(cells[0])
+                    if fam and cells[3] == cur[fam]:
+                        out[(cells[0], int(cells[1]))] = int(cells[2])
     except OSError:
         pass
     return out
@@ -616,7 +626,12 @@ def main():
                     help="run a few eager quant + GEMM launches of one workload and exit (for ncu)")
     ap.add_argument("--profile-m", type=int, default=None)
     ap.add_argument("--profile-iters", type=int, default=4)
+    ap.add_argument("--kernel-hashes", action="store_true",
+                    help="print the source hash of each kernel family (the key of profiles/traffic.md rows) and exit")
     args = ap.parse_args()
+    if args.kernel_hashes:
+        print(json.dumps({fam: kernel_hash(fam) for fam in KERNEL_FAMILIES}))
+        return
 
     rank, world, local = dist_init()
     try:

@@ -310,8 +310,10 @@ MX_API mx_status mx_gemm_grouped(const void* a_codes, const void* a_scales, mx_a
  * word is used (calls never keep split-K partials there), so decode-sized
  * problems take the cluster-reduced split plan.  The call allocates and
  * frees nothing.  Its first call on a device looks the array's device address
- * up once (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture.  All calls share the array, which keeps what
+ * up (cudaGetSymbolAddress, with that device current) and keeps it for that
+ * device's context; make that first call before any stream capture, and again
+ * after a device reset or anything else that replaces the context, which
+ * looks the address up anew.  All calls share the array, which keeps what
  * the last call left there (only a give-up of a bounded wait writes it, and no
  * kernel reads it back), so calls that overlap on the GPU race on it.  A
  * give-up cannot be read back through this call; use mx_gemm with a workspace

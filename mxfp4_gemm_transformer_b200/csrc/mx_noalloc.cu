@@ -8,6 +8,9 @@
 // device allocator at all.  mx_gemm_noalloc serves them: it takes the same
 // inputs and outputs and uses a scratch array that lives in the library
 // itself, so the call allocates nothing.
+#include <cuda.h>
+
+#include <cstdint>
 #include <mutex>
 
 #include "mx_internal.h"
@@ -19,23 +22,56 @@ namespace {
 // loads the library holds these bytes until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MX_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch, resolved once per device with that
-// device current (in host code the symbol's name is only a host-side stand-in,
-// never a device address).
+// Identity of the current context: its unique id where the driver has
+// cuCtxGetId (a destroyed and recreated context gets a new one, even at the
+// same address), else the context handle; 0 when neither can be read.
+unsigned long long context_identity()
+{
+    using GetCurrentFn = CUresult (*)(CUcontext*);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    if (get_id && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+    return static_cast<unsigned long long>(reinterpret_cast<uintptr_t>(ctx));
+}
+
+// Device address of g_noalloc_scratch, resolved with the device current (in
+// host code the symbol's name is only a host-side stand-in, never a device
+// address) and cached per device together with the context it belongs to: a
+// device reset, or a new primary context, loads the module again and may move
+// the array, so a changed context is looked up afresh.
 cudaError_t scratch_address(void** out)
 {
     static std::mutex mu;
     static void* addr[64] = {};
+    static unsigned long long owner[64] = {};
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const unsigned long long ctx = context_identity();
     std::lock_guard<std::mutex> lk(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || ctx == 0 || owner[dev] != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
         addr[dev] = p;
+        owner[dev] = ctx;
     }
     *out = addr[dev];
     return cudaSuccess;
