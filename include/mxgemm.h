@@ -387,14 +387,12 @@ MX_API void mx_set_launch_flags(unsigned flags);
 
 /*
  * mx_set_decode_tuning -- process-wide override of the decode kernel choice,
- * for tuning and tests.  There are two decode kernels: weights on the MMA's
- * 128-row side (any format), and weights on its N side (240 weight rows per
- * MMA; E8M0 formats, cluster or whole-tile splits; measured slower, so only
- * on request).  mode 0: automatic (the 128-row-side kernel for M <= 64, unless
- * mx_set_tuning overrides are set); 1: the 128-row-side kernel whenever it can
- * run the problem (M <= 64; K % 128 == 0 for E8M0 formats), even with
- * mx_set_tuning overrides or few tiles; 2: the N-side kernel whenever it can,
- * else as 1; -1: neither.
+ * for tuning and tests.  The decode kernel puts the weights on the MMA's
+ * 128-row side and the tokens on its N side.  mode 0: automatic (the decode
+ * kernel for M <= 64, unless mx_set_tuning overrides are set); 1 (or more):
+ * the decode kernel whenever it can run the problem (M <= 64; K % 128 == 0
+ * for E8M0 formats), even with mx_set_tuning overrides or few tiles; -1:
+ * never.
  * ctas: its grid size (0 = one CTA per SM).  ctas_per_sm: its shared-memory
  * budget -- 2 (at most 113 KB, so the next launch's CTAs can start beside this
  * launch's), 1 (a deep weight ring for long-running problems), 0 = choose.
@@ -406,8 +404,8 @@ MX_API void mx_set_launch_flags(unsigned flags);
  * distributed shared memory, in rank order), 2 stream-K (equal ranges of
  * (tile, K block) units over `ctas` CTAs; cut tiles reduced with fp32 atomic
  * adds in the workspace, arrival order), 3 whole tiles.  cluster_size: CTAs
- * per cluster for split 0 / 1 (2..8, up to 16 for the N-side kernel; 0 = fill
- * the SMs).  Not for concurrent use with other threads' mx_gemm calls.
+ * per cluster for split 0 / 1 (2..8; 0 = fill the SMs).  Not for concurrent
+ * use with other threads' mx_gemm calls.
  */
 MX_API void mx_set_decode_tuning(int mode, int ctas, int ctas_per_sm, int prefetch_stages, int split,
                                  int cluster_size);
@@ -448,11 +446,10 @@ MX_API mx_status mx_gemm_plan(int M, int N, int K, mx_a_fmt a_fmt, mx_b_fmt b_fm
 typedef struct mx_plan_info {
     int kernel;      /* 0: tile kernel (activation-row x weight-row tiles);
                         1: decode kernel (weights as the MMA's 128-row side);
-                        2: decode kernel (weights as the MMA's N side);
                         3: tile kernel over CTA pairs (256 x 240 tiles,
                            cta_group::2 MMAs) */
     int block_m;     /* activation rows per tile (decode kernel: tokens per MMA) */
-    int block_n;     /* weight rows per tile (decode kernels: 128 per sub-tile, or 240) */
+    int block_n;     /* weight rows per tile (decode kernel: 128 per sub-tile) */
     int splits;      /* K splits per tile (decode kernel: about how many CTAs
                         share one tile) */
     int k_reduction; /* 0 none; 1 thread-block cluster (distributed shared

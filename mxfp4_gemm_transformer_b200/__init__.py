@@ -227,8 +227,7 @@ def mx_gemm_plan_info(M, N, K, a_fmt, b_fmt, epi, ws_bytes=None):
     wsb = ctypes.c_size_t(-1).value if ws_bytes is None else ws_bytes
     _check(load().mx_gemm_plan_info(M, N, K, a_fmt, b_fmt, epi, wsb, ctypes.byref(info)), "mx_gemm_plan_info")
     d = {name: getattr(info, name) for name, _ in PlanInfo._fields_}
-    d["kernel"] = {1: "decode", 2: "decode", 3: "pair"}.get(info.kernel, "tile")
-    d["weights_on"] = {1: "M", 2: "N"}.get(info.kernel)
+    d["kernel"] = {1: "decode", 3: "pair"}.get(info.kernel, "tile")
     d["k_reduction"] = K_REDUCTION.get(info.k_reduction, str(info.k_reduction))
     return d
 

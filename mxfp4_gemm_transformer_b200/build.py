@@ -21,7 +21,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmxgemm.so")
 TRACE_LIB = os.path.join(HERE, "libmxgemm_trace.so")
 SOURCES = ["mx_api.cu", "mx_quant.cu", "mx_norm_quant.cu", "mx_gemm.cu", "mx_gemm_pair.cu", "mx_decode.cu",
-           "mx_decode_nw.cu", "mx_noalloc.cu"]
+           "mx_noalloc.cu"]
 DEPS = ["mx_internal.h", "mx_ptx.cuh", "mx_kernel_common.cuh", "mx_quant_common.cuh", "mx_decode_common.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 

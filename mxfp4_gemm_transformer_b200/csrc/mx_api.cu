@@ -264,10 +264,10 @@ void mx_set_launch_flags(unsigned flags)
 
 void mx_set_decode_tuning(int mode, int ctas, int ctas_per_sm, int prefetch_stages, int split, int cluster_size)
 {
-    set_decode_tuning(mode < 0 ? -1 : (mode > 2 ? 0 : mode), ctas < 0 ? 0 : ctas,
+    set_decode_tuning(mode < 0 ? -1 : (mode > 0 ? 1 : 0), ctas < 0 ? 0 : ctas,
                       (ctas_per_sm == 1 || ctas_per_sm == 2) ? ctas_per_sm : 0,
                       prefetch_stages < 0 ? 0 : prefetch_stages, (split >= 0 && split <= 3) ? split : 0,
-                      (cluster_size >= 2 && cluster_size <= 16) ? cluster_size : 0);
+                      (cluster_size >= 2 && cluster_size <= 8) ? cluster_size : 0);
 }
 
 mx_status mx_gemm_plan_info(int M, int N, int K, mx_a_fmt a_fmt, mx_b_fmt b_fmt, mx_epi epi, size_t ws_bytes,
@@ -292,7 +292,7 @@ mx_status mx_gemm_plan_info(int M, int N, int K, mx_a_fmt a_fmt, mx_b_fmt b_fmt,
     info->block_m = plan.block_m;
     info->block_n = plan.block_n;
     info->splits = plan.splits;
-    if (plan.kernel == 1 || plan.kernel == 2)
+    if (plan.kernel == 1)
         info->k_reduction = plan.reduce ? 3 : (plan.cluster > 1 ? 1 : 0);
     else
         info->k_reduction = plan.splits > 1 ? (plan.gsplit ? 2 : 1) : 0;
@@ -301,7 +301,7 @@ mx_status mx_gemm_plan_info(int M, int N, int K, mx_a_fmt a_fmt, mx_b_fmt b_fmt,
     info->stages = plan.stages;
     info->tiles = plan.kernel != 0 ? plan.tiles : plan.units / std::max(1, plan.splits);
     info->ws_bytes = std::max(plan.ws_bytes, kWorkspaceBytes);
-    info->ctas_per_sm = (plan.kernel == 1 || plan.kernel == 2) ? (plan.one_per_sm ? 1 : 2) : 1;
+    info->ctas_per_sm = plan.kernel == 1 ? (plan.one_per_sm ? 1 : 2) : 1;
     info->act_quant = plan.act_quant;
     return MX_OK;
 }

@@ -1,7 +1,6 @@
-// mx_decode_common.cuh -- what the two decode kernels (weights on the MMA's
-// 128-row side, mx_decode.cu; weights on its N side, mx_decode_nw.cu) share:
-// the launch arguments, the trace stamps, the epilogue value of one output
-// and the fused quantisation of bf16 tokens into the token ring.
+// mx_decode_common.cuh -- parts of the decode kernel (mx_decode.cu): the
+// launch arguments, the trace stamps, the epilogue value of one output and the
+// fused quantisation of bf16 tokens into the token ring.
 #pragma once
 #include <cuda_bf16.h>
 

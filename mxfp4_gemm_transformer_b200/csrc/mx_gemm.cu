@@ -1266,7 +1266,7 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
         q.a_fmt = MX_A_E4M3_E8M0_1X32;
         cudaError_t e = plan_gemm(q, dev, ws_bytes, plan);
         if (e != cudaSuccess) return e;
-        const bool fusable = plan->kernel == 1 || plan->kernel == 2;  // both decode kernels quantise tokens
+        const bool fusable = plan->kernel == 1;  // the decode kernel quantises tokens
         if (fusable && static_cast<long long>(pb.M) * plan->tiles <= kFusedQuantMaxWork) {
             plan->act_quant = 1;
             return cudaSuccess;
@@ -1291,7 +1291,6 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
     }
     const bool swiglu = epi_swiglu(pb.epi);
     const int sc = pb.a_fmt == MX_A_E4M3_E8M0_1X32 ? 1 : (pb.a_fmt == MX_A_E2M1_E8M0_1X32 ? 2 : 0);
-    const bool scaled = sc != 0;
     const int nout = swiglu ? pb.N / 2 : pb.N;
     const int num_kb = (pb.K + 127) / 128;
     const int tiles_m = (pb.M + 127) / 128;
@@ -1317,36 +1316,6 @@ cudaError_t plan_gemm(const GemmProblem& pb, const DeviceInfo& dev, size_t ws_by
     const bool tuned = g_tune_bn != 0 || g_tune_splits != 0 || g_tune_bm != 0 || g_tune_ctas != 0;
     if (pb.M <= 64 && g_dec_mode >= 0 && (g_dec_mode >= 1 || !tuned) && sc != 2) {
         const bool det = (launch_flags() & MX_LAUNCH_DETERMINISTIC) != 0;
-        // On request (mode 2), for E8M0 formats: the kernel with the weights
-        // on the MMA's N side (240 weight rows per instruction, 1.9x the
-        // weight bytes of the 128-row side at the same issue cost), split like
-        // the other below but with clusters of up to 16; stream-K stays with
-        // the other kernel.  Not the default: with only M of its 128 token
-        // lanes real, its epilogue and cluster reduction run on one or two
-        // warps, and it measured slower on every decode workload (e.g. the
-        // fused q_a + kv shape at M = 1: 8.0 against 7.0 us; W4A8 gate_up at
-        // M = 16: 27.8 against 23.5 us).
-        if (g_dec_mode == 2 && g_dec_split != kDecStreamK) {
-            const int out_nw = swiglu ? 120 : 240;
-            const int tiles_nw = ((swiglu ? pb.N / 2 : pb.N) + out_nw - 1) / out_nw;
-            const bool short_nw = tiles_nw * 2 <= sms;
-            const int grid_nw = g_dec_ctas > 0 ? g_dec_ctas : (short_nw ? sms : 2 * sms);
-            const int per_sm_nw = g_dec_per_sm > 0 ? g_dec_per_sm : 2;
-            const int cl = g_dec_cluster > 0 ? g_dec_cluster
-                                             : std::min(16, (short_nw ? sms : 2 * sms) / std::max(1, tiles_nw));
-            GemmPlan np;
-            if ((g_dec_split == kDecAuto || g_dec_split == kDecCluster) && cl >= 2 &&
-                tiles_nw * cl <= 2 * sms && plan_decode_nw(pb, kDecCluster, grid_nw, cl, per_sm_nw, &np)) {
-                *plan = np;
-                return cudaSuccess;
-            }
-            np = GemmPlan();
-            if (g_dec_split != kDecCluster && plan_decode_nw(pb, kDecWholeTiles, grid_nw, 1, per_sm_nw, &np) &&
-                (np.grid_x * 10 >= sms * 8 || g_dec_split == kDecWholeTiles || g_dec_mode == 2)) {
-                *plan = np;
-                return cudaSuccess;
-            }
-        }
         const int nout_d = swiglu ? pb.N / 2 : pb.N;
         const int tiles_d = (nout_d + 127) / 128;
         const bool short_launch = tiles_d * 2 <= sms;
@@ -1577,7 +1546,6 @@ cudaError_t launch_gemm(const GemmProblem& pb, const GemmPlan& plan, cudaStream_
         return launch_quant_e8m0_1x32(tmp, pb.M, pb.N / 2, codes, codes + static_cast<size_t>(pb.M) * (pb.N / 2), st);
     }
     if (plan.kernel == 1) return launch_decode(pb, plan, st);
-    if (plan.kernel == 2) return launch_decode_nw(pb, plan, st);
     if (plan.kernel == 3) return launch_pair(pb, plan, st);
     const bool swiglu = epi_swiglu(pb.epi);
     const int sc = pb.a_fmt == MX_A_E4M3_E8M0_1X32 ? 1 : (pb.a_fmt == MX_A_E2M1_E8M0_1X32 ? 2 : 0);

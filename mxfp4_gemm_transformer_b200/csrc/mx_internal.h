@@ -107,8 +107,7 @@ struct GemmPlan {
     int stages = 0;       // shared-memory ring depth
     // decode kernel (kernel == 1): weights are the MMA's 128-row side, tokens its N
     int kernel = 0;       // 0 = tile kernel (mx_gemm.cu), 1 = decode kernel, weights on the MMA's M side
-                          // (mx_decode.cu), 2 = decode kernel, weights on its N side (mx_decode_nw.cu),
-                          // 3 = tile kernel over CTA pairs (mx_gemm_pair.cu)
+                          // (mx_decode.cu), 3 = tile kernel over CTA pairs (mx_gemm_pair.cu)
     int tiles = 0;        // decode: tiles of 128 output columns
     int whole_tiles = 0;  // decode: CTAs take whole tiles (no cross-CTA reduction)
     int reduce = 0;       // decode: some tile's K range is split between CTAs (workspace accumulators)
@@ -162,8 +161,6 @@ int decode_tokens_tile(int M, bool short_launch);
 size_t decode_ws_bytes(int tiles, int nsub, int M);
 bool plan_decode(const GemmProblem& pb, int split, int grid, int cluster, int per_sm, int sms, GemmPlan* plan);
 cudaError_t launch_decode(const GemmProblem& pb, const GemmPlan& plan, cudaStream_t st);
-bool plan_decode_nw(const GemmProblem& pb, int split, int grid, int cluster, int per_sm, GemmPlan* plan);
-cudaError_t launch_decode_nw(const GemmProblem& pb, const GemmPlan& plan, cudaStream_t st);
 void set_timeline(void* buf, size_t bytes);
 constexpr int kTimelineCtaSlots = 16;  // per-CTA records ahead of the 4 x 64 per-stage detail
 unsigned long long* timeline_buffer(int* ctas);  // installed trace buffer (null = off)

@@ -41,9 +41,9 @@ WORKLOADS = [
 def plan_tiles(plan, M, swiglu):
     """(rows per tile, output columns per tile) of the plan that ran."""
     if plan["kernel"] == "decode":
-        # one tile of tokens; 128 weight rows (or 240 on the MMA's N side) per
-        # output tile, a gate and an up sub-tile of 128 each for SwiGLU
-        return M, (128 if plan["weights_on"] == "M" else (120 if swiglu else 240))
+        # one tile of tokens; 128 weight rows per output tile, a gate and an
+        # up sub-tile of 128 each for SwiGLU
+        return M, 128
     bn = plan["block_n"]
     return plan["block_m"], (bn // 2 if swiglu else bn)
 

@@ -2,10 +2,9 @@
 the ViT page's `vt_add` update x += y + b fused into the GEMM) against the
 oracle's gemm_residual, element by element within
 |y_gpu - y| <= 2^-8 |y| + 1e-5 T, on every kernel and plan: the decode kernel
-(cluster, whole tiles, stream-K), the decode kernel with the weights on the
-MMA's N side, the tile kernel with 128- and 256-row tiles, K split through the
-workspace or over a cluster, and the CTA-pair kernel; with and without a
-bias; ragged M and N."""
+(cluster, whole tiles, stream-K), the tile
+kernel with 128- and 256-row tiles, K split through the workspace or over a
+cluster, and the CTA-pair kernel; with and without a bias; ragged M and N."""
 import numpy as np
 import pytest
 import torch
@@ -44,7 +43,6 @@ PLANS = [
     ("decode-cluster", dict(decode=1, split=1, cluster=4), "min"),
     ("decode-whole", dict(decode=1, split=3), "min"),
     ("decode-streamk", dict(decode=1, split=2), "full"),
-    ("decode-nw", dict(decode=2, split=1, cluster=4), "min"),
     ("tile-128", dict(decode=-1, block_n=240, splits=1, block_m=128), "full"),
     ("tile-256", dict(decode=-1, block_n=240, splits=1, block_m=256), "full"),
     ("tile-splitk-ws", dict(decode=-1, block_n=128, splits=4), "full"),
