@@ -90,7 +90,12 @@ struct DecCfg {
     static_assert(DW * W_BYTES >= NSUB * MT * 128 * 4, "the weight ring holds a cluster partial");
 };
 
-template <int MT, int NSUB, bool SCALED, bool ONE_PER_SM>
+// CL: the instance for cluster splits (a tile's K range over the CTAs of a
+// thread-block cluster, partials reduced in distributed shared memory); the
+// other instance runs whole tiles and stream-K.  Each carries only its own
+// epilogue: on these microsecond launches the code on the critical path is
+// fetched cold, so code that a launch never runs still costs time.
+template <int MT, int NSUB, bool SCALED, bool ONE_PER_SM, bool CL>
 __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel(const __grid_constant__ DecodeArgs p)
 {
     using C = DecCfg<MT, NSUB, SCALED, ONE_PER_SM>;
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
 
     // this CTA's units [g0, g1) (unit = tile * num_kb + K block)
     int g0, g1;
-    const int S = p.cluster_s;
+    const int S = CL ? p.cluster_s : 1;
     const int crank = S > 1 ? static_cast<int>(cluster_ctarank()) : 0;
     if (S > 1) {
         // one tile per cluster; rank r takes K blocks [r nkb / S, (r + 1) nkb / S)
@@ -476,6 +481,7 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
             }
             g = g1;  // no per-segment epilogue below
         }
+        if constexpr (!CL)
         while (g < g1) {
             const int tile = g / p.num_kb;
             const int kb0 = g - tile * p.num_kb;
@@ -757,11 +763,11 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
 
 namespace {
 
-template <int MT, int NSUB, bool SCALED, bool ONE>
+template <int MT, int NSUB, bool SCALED, bool ONE, bool CL>
 cudaError_t prepare_decode()
 {
     using C = DecCfg<MT, NSUB, SCALED, ONE>;
-    auto kern = decode_kernel<MT, NSUB, SCALED, ONE>;
+    auto kern = decode_kernel<MT, NSUB, SCALED, ONE, CL>;
     static std::mutex mu;
     static bool done[64] = {};
     int dev = 0;
@@ -783,11 +789,11 @@ struct DecLaunch {
     int grid;
     int cluster;
     cudaStream_t st;
-    template <int MT, int NSUB, bool SCALED, bool ONE>
+    template <int MT, int NSUB, bool SCALED, bool ONE, bool CL>
     cudaError_t run() const
     {
         using C = DecCfg<MT, NSUB, SCALED, ONE>;
-        cudaError_t e = prepare_decode<MT, NSUB, SCALED, ONE>();
+        cudaError_t e = prepare_decode<MT, NSUB, SCALED, ONE, CL>();
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(grid, 1, 1);
@@ -810,7 +816,7 @@ struct DecLaunch {
         }
         cfg.attrs = attr;
         cfg.numAttrs = na;
-        return cudaLaunchKernelEx(&cfg, decode_kernel<MT, NSUB, SCALED, ONE>, *args);
+        return cudaLaunchKernelEx(&cfg, decode_kernel<MT, NSUB, SCALED, ONE, CL>, *args);
     }
     cudaError_t invalid() const { return cudaErrorInvalidValue; }
 };
@@ -819,7 +825,7 @@ struct DecLaunch {
 // (cached per device, variant and size; 0 when the query fails).
 struct DecClusters {
     int cluster;
-    template <int MT, int NSUB, bool SCALED, bool ONE>
+    template <int MT, int NSUB, bool SCALED, bool ONE, bool CL>
     int run() const
     {
         using C = DecCfg<MT, NSUB, SCALED, ONE>;
@@ -831,7 +837,7 @@ struct DecClusters {
             std::lock_guard<std::mutex> lk(mu);
             if (cache[dev][cluster]) return cache[dev][cluster] > 0 ? cache[dev][cluster] : 0;
         }
-        if (prepare_decode<MT, NSUB, SCALED, ONE>() != cudaSuccess) return 0;
+        if (prepare_decode<MT, NSUB, SCALED, ONE, CL>() != cudaSuccess) return 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(cluster * 16, 1, 1);
         cfg.blockDim = dim3(kDecThreads, 1, 1);
@@ -844,7 +850,7 @@ struct DecClusters {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<MT, NSUB, SCALED, ONE>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<MT, NSUB, SCALED, ONE, CL>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -856,30 +862,36 @@ struct DecClusters {
 };
 
 struct DecStages {
-    template <int MT, int NSUB, bool SCALED, bool ONE>
+    template <int MT, int NSUB, bool SCALED, bool ONE, bool CL>
     int run() const { return DecCfg<MT, NSUB, SCALED, ONE>::DW; }
     int invalid() const { return 0; }
 };
 
 struct DecAccBufs {
-    template <int MT, int NSUB, bool SCALED, bool ONE>
+    template <int MT, int NSUB, bool SCALED, bool ONE, bool CL>
     int run() const { return DecCfg<MT, NSUB, SCALED, ONE>::ACC_BUFS; }
     int invalid() const { return 0; }
 };
 
 template <class Op>
-auto dec_dispatch(int mt, bool swiglu, bool scaled, bool one, const Op& op) -> decltype(op.invalid())
+auto dec_dispatch(int mt, bool swiglu, bool scaled, bool one, bool cl, const Op& op) -> decltype(op.invalid())
 {
-#define MXG_DEC(T, O)                                                                                       \
-    if (mt == T && one == O)                                                                                \
-        return swiglu ? (scaled ? op.template run<T, 2, true, O>() : op.template run<T, 2, false, O>())     \
-                      : (scaled ? op.template run<T, 1, true, O>() : op.template run<T, 1, false, O>());
-    MXG_DEC(16, false)
-    MXG_DEC(32, false)
-    MXG_DEC(64, false)
-    MXG_DEC(16, true)
-    MXG_DEC(32, true)
-    MXG_DEC(64, true)
+#define MXG_DEC(T, O, L)                                                                                          \
+    if (mt == T && one == O && cl == L)                                                                           \
+        return swiglu ? (scaled ? op.template run<T, 2, true, O, L>() : op.template run<T, 2, false, O, L>())     \
+                      : (scaled ? op.template run<T, 1, true, O, L>() : op.template run<T, 1, false, O, L>());
+    MXG_DEC(16, false, false)
+    MXG_DEC(32, false, false)
+    MXG_DEC(64, false, false)
+    MXG_DEC(16, true, false)
+    MXG_DEC(32, true, false)
+    MXG_DEC(64, true, false)
+    MXG_DEC(16, false, true)
+    MXG_DEC(32, false, true)
+    MXG_DEC(64, false, true)
+    MXG_DEC(16, true, true)
+    MXG_DEC(32, true, true)
+    MXG_DEC(64, true, true)
 #undef MXG_DEC
     return op.invalid();
 }
@@ -943,8 +955,8 @@ bool plan_decode(const GemmProblem& pb, int split, int grid, int cluster, int pe
         per_cta = (total + g - 1) / g;
     }
     bool one = per_sm == 1;
-    if (per_sm == 0) one = per_cta > 3LL * dec_dispatch(mt, swiglu, scaled, false, DecStages{});
-    if (S > 1 && dec_dispatch(mt, swiglu, scaled, one, DecClusters{S}) < 1) return false;
+    if (per_sm == 0) one = per_cta > 3LL * dec_dispatch(mt, swiglu, scaled, false, false, DecStages{});
+    if (S > 1 && dec_dispatch(mt, swiglu, scaled, one, true, DecClusters{S}) < 1) return false;
     plan->kernel = 1;
     plan->block_n = 128;
     plan->block_m = mt;
@@ -966,8 +978,8 @@ bool plan_decode(const GemmProblem& pb, int split, int grid, int cluster, int pe
     plan->gsplit = 0;
     plan->part_rows = 0;
     plan->ws_bytes = cut ? decode_ws_bytes(tiles, nsub, pb.M) : kWorkspaceHeader;
-    plan->acc_bufs = dec_dispatch(mt, swiglu, scaled, one, DecAccBufs{});
-    plan->stages = dec_dispatch(mt, swiglu, scaled, one, DecStages{});
+    plan->acc_bufs = dec_dispatch(mt, swiglu, scaled, one, false, DecAccBufs{});
+    plan->stages = dec_dispatch(mt, swiglu, scaled, one, false, DecStages{});
     return true;
 }
 
@@ -1039,7 +1051,8 @@ cudaError_t launch_decode(const GemmProblem& pb, const GemmPlan& plan, cudaStrea
     // 64 bytes in memory, 128 in shared memory)
     const uint32_t w_row_bytes = e2m1 ? 64u : 128u;
     a.w_tx = static_cast<uint32_t>(swiglu ? 2 : 1) * 128u * w_row_bytes;
-    return dec_dispatch(mt, swiglu, scaled, plan.one_per_sm != 0, DecLaunch{&a, plan.grid_x, a.cluster_s, st});
+    return dec_dispatch(mt, swiglu, scaled, plan.one_per_sm != 0, a.cluster_s > 1,
+                        DecLaunch{&a, plan.grid_x, a.cluster_s, st});
 }
 
 }  // namespace mxg
