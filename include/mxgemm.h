@@ -25,7 +25,8 @@
  *   - All matrix pointers are DEVICE pointers owned by the caller; dense,
  *     row-major, no padding between rows.  The library allocates nothing,
  *     never synchronises the device (except mx_workspace_status) and launches
- *     only on the given stream, so the calls can be captured in a CUDA graph.
+ *     only on the given stream, so the calls that take a workspace can be
+ *     captured in a CUDA graph.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
  *   - Every pointer must be 16-byte aligned; e2m1 weight codes 32-byte aligned.
  *   - Errors found while validating return at once and launch nothing.  A
@@ -296,10 +297,9 @@ MX_API mx_status mx_gemm_grouped(const void* a_codes, const void* a_scales, mx_a
 /*
  * mx_gemm_noalloc -- mx_gemm for callers that cannot allocate device memory.
  * The pages have no counterpart to this call; it exists for users of this
- * library who cannot hand mx_gemm a workspace: code running while a stream is
- * captured (cudaMalloc is no stream operation and synchronises the device),
- * runtimes that give kernels a fixed arena and forbid hidden allocations, and
- * plain-C plugin hosts with no device allocator.
+ * library who cannot hand mx_gemm a workspace: runtimes that give kernels a
+ * fixed arena and forbid hidden allocations, and plain-C plugin hosts with no
+ * device allocator.
  *
  * Same arguments, results and tolerance as mx_gemm, minus the workspace.  The
  * scratch is a MX_NOALLOC_SCRATCH_BYTES array inside the library, held by
@@ -311,9 +311,8 @@ MX_API mx_status mx_gemm_grouped(const void* a_codes, const void* a_scales, mx_a
  * problems take the cluster-reduced split plan.  The call allocates and
  * frees nothing.  Its first call on a device looks the array's device address
  * up (cudaGetSymbolAddress, with that device current) and keeps it for that
- * device's context; make that first call before any stream capture, and again
- * after a device reset or anything else that replaces the context, which
- * looks the address up anew.  All calls share the array, which keeps what
+ * device's context; after a device reset or anything else that replaces the
+ * context, the next call looks the address up anew.  All calls share the array, which keeps what
  * the last call left there (only a give-up of a bounded wait writes it, and no
  * kernel reads it back), so calls that overlap on the GPU race on it.  A
  * give-up cannot be read back through this call; use mx_gemm with a workspace

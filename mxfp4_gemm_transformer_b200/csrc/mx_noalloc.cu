@@ -1,11 +1,9 @@
 // mx_noalloc.cu -- mx_gemm for callers that cannot allocate device memory.
 //
 // mx_gemm needs a small caller-owned workspace (the status word its bounded
-// waits report into).  Some callers have no way to provide one: code that runs
-// while a stream is being captured (cudaMalloc is not a stream operation and
-// synchronises the device), runtimes that hand kernels a fixed memory arena
-// and forbid hidden allocations, and plain-C plugin hosts that expose no
-// device allocator at all.  mx_gemm_noalloc serves them: it takes the same
+// waits report into).  Some callers have no way to provide one: runtimes that
+// hand kernels a fixed memory arena and forbid hidden allocations, and plain-C
+// plugin hosts that expose no device allocator at all.  mx_gemm_noalloc serves them: it takes the same
 // inputs and outputs and uses a scratch array that lives in the library
 // itself, so the call allocates nothing.
 #include <cuda.h>

@@ -1,7 +1,7 @@
 """mx_gemm_noalloc: the GEMM for callers that cannot allocate device memory.
 
-Callers inside stream capture, with a fixed memory arena, or behind a C plugin
-interface without a device allocator cannot give mx_gemm its workspace; this
+Callers with a fixed memory arena, or behind a C plugin interface without a
+device allocator, cannot give mx_gemm its workspace; this
 entry point uses scratch that lives in the library instead.  The test calls it
 through the C ABI twice in a row and checks each result against mx_gemm's on
 the same inputs, with the acceptance bound the other GEMM tests use.  The file
