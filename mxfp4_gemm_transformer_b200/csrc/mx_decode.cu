@@ -154,8 +154,8 @@ __global__ void __launch_bounds__(kDecThreads, ONE_PER_SM ? 1 : 2) decode_kernel
             mbar_init(&wfull[s], SCALED ? 1 + 32 : 1);
             mbar_init(&wempty[s], 1);
         }
-        // one arrival per lane of the token producer, or per quantising thread
-        const uint32_t x_arrivals = (SCALED && p.x_bf16) ? 32u * static_cast<uint32_t>(p.xq_warps) : 32u;
+        // one arrival per lane of the token producer, or per quantising warp
+        const uint32_t x_arrivals = (SCALED && p.x_bf16) ? static_cast<uint32_t>(p.xq_warps) : 32u;
         for (int s = 0; s < C::DX; ++s) {
             mbar_init(&xfull[s], x_arrivals);
             mbar_init(&xempty[s], 1);

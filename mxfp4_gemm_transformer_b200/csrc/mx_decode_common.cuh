@@ -127,10 +127,10 @@ __device__ __forceinline__ void dec_store_mxq(const DecodeArgs& p, int m, int j,
 // units belong to different threads and their loads are in flight together.
 // Each thread keeps its next two blocks loaded ahead of their conversion and
 // walks the units in order: it waits until the unit's ring stage is free,
-// writes its blocks of that unit, fences them to the tensor core's (async)
-// proxy and arrives on the stage's barrier (every thread arrives for every
-// unit, which also keeps each thread within one phase of every stage's
-// barriers).  Rows >= M are not written: an MMA output column depends on its
+// writes its blocks of that unit and fences them to the tensor core's (async)
+// proxy; then its warp arrives once on the stage's barrier (every warp
+// arrives for every unit, which also keeps each thread within one phase of
+// every stage's barriers).  All 32 lanes of each quantising warp call this.  Rows >= M are not written: an MMA output column depends on its
 // own token row alone and columns >= M are never stored.
 template <class C>
 __device__ __forceinline__ void dec_load_block(const DecodeArgs& p, int g0, int b, uint4 (&v)[4])
@@ -195,7 +195,7 @@ __device__ __forceinline__ void dec_quant_tokens(const DecodeArgs& p, int g0, in
     }
     uint32_t xs = 0, xph = 0;
     for (int i = 0; i < n_units; ++i) {
-        if (!wait_bar(&xempty[xs], xph ^ 1u, abort_flag, p.status)) break;
+        if (__any_sync(0xFFFFFFFFu, !wait_bar(&xempty[xs], xph ^ 1u, abort_flag, p.status))) break;
         uint8_t* xt = xring + xs * C::X_BYTES;
         uint8_t* sf = sfb_ring + xs * C::SFB_BYTES;
         while (b0 < total && b0 / per_unit == i) {
@@ -210,8 +210,11 @@ __device__ __forceinline__ void dec_quant_tokens(const DecodeArgs& p, int g0, in
                 nb += nthreads;
             }
         }
+        // every lane's writes to the async proxy, then one arrival per warp
+        // (one per lane serialised on the barrier measured ~1 us per launch)
         fence_proxy_async_smem();
-        mbar_arrive(&xfull[xs]);
+        __syncwarp();
+        if ((qid & 31) == 0) mbar_arrive(&xfull[xs]);
         if (++xs == C::DX) {
             xs = 0;
             xph ^= 1u;
